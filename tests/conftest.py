@@ -1,0 +1,30 @@
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+    config.addinivalue_line("markers", "slow: full-size workload check")
+
+
+@pytest.fixture(scope="session", autouse=True)
+def _built_helpers():
+    # the CPU oracle and the input generator are plain C; build them if missing
+    import oracle
+    import synth
+
+    oracle.build()
+    synth.build()
+    yield
+
+
+def has_gpu() -> bool:
+    import torch
+
+    return torch.cuda.is_available()
