@@ -1,0 +1,196 @@
+/*
+ * moe.h — C ABI of libmoe.so: forward pass of one Mixture-of-Experts
+ * feed-forward layer on one NVIDIA B200 (sm_100a).
+ *
+ *   R = X + MoE(RMSNorm(X))
+ *
+ * Sources (web pages on MoE inference; each entry point cites its passage):
+ *   [P1] "推理计算流梳理" (huanyp.cn) — §Norm&Residual, §实际 MLP 计算策略,
+ *        §专家并行 / MoE Router 过程, §EP 路径.
+ *   [P5] "「赤兔」Chitu 框架深度解读（七）：混合专家模型 (MoE) 的高效处理" —
+ *        §Token 分发策略 (MoETokenDispatcher: token_permutation /
+ *        token_unpermutation), §专家计算实现 (BatchedExperts; tokens laid out
+ *        contiguously by expert id for the grouped GEMM).
+ *
+ * Conventions shared by every entry point
+ *   - Pointers named as tensors are DEVICE pointers owned by the caller; the
+ *     library never allocates, frees or keeps them.  Host pointers are only
+ *     the small structs (moe_shape_t, moe_weights_t) and size_t* ws_bytes.
+ *   - Layouts are row-major with the last index contiguous.  Weights are
+ *     stored out x in: W_r [E][d], W_gate/W_up [E][d_ff][d], W_down [E][d][d_ff].
+ *   - Work is queued on `stream` and never synchronised with the host.
+ *   - Workspace: pass ws == NULL to have the size needed written to *ws_bytes
+ *     (returns MOE_OK, queues nothing).  A buffer smaller than needed gives
+ *     MOE_ERR_WORKSPACE with the needed size in *ws_bytes.  ws must be 256-byte
+ *     aligned and must not be used by other work until the queued work ends.
+ *   - Arguments are validated on the host before anything is queued; on any
+ *     error nothing is queued.  No entry point throws, aborts or prints.
+ *   - Errors found by kernels (bad expert ids, a bounded wait that gave up)
+ *     are OR-ed as MOE_DEV_* bits into *dev_status when dev_status != NULL.
+ *   - T == 0 is valid and queues nothing (moe_forward still clears dev_status).
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t (NULL = the legacy default stream). */
+typedef struct CUstream_st* moe_stream_t;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1, /* null pointer, negative or inconsistent size, misaligned pointer */
+    MOE_ERR_UNSUPPORTED = 2, /* well-formed but outside what the kernels support (see each call) */
+    MOE_ERR_WORKSPACE = 3,   /* workspace too small; *ws_bytes holds the size needed */
+    MOE_ERR_CUDA = 4,        /* a CUDA runtime call or a kernel launch failed */
+    MOE_ERR_DEVICE = 5       /* the current device is not sm_100 */
+} moe_status_t;
+
+/* bits OR-ed into *dev_status by kernels */
+#define MOE_DEV_BAD_EXPERT_ID 1 /* topk_idx held an id outside [0, E); that pair was dropped */
+#define MOE_DEV_TIMEOUT 2       /* a bounded in-kernel wait gave up; outputs are not valid */
+
+#define MOE_MAX_EXPERTS 256
+#define MOE_MAX_TOP_K 8
+
+typedef struct {
+    int32_t T;     /* tokens (rows of X) */
+    int32_t d;     /* hidden size */
+    int32_t E;     /* experts */
+    int32_t top_k; /* experts per token, 1..8 */
+    int32_t d_ff;  /* expert hidden size */
+    float eps;     /* RMSNorm epsilon */
+    moe_dtype_t x_dtype;   /* X and the residual */
+    moe_dtype_t w_dtype;   /* expert weights (bf16: tensor-core path; f32: CUDA-core path) */
+    moe_dtype_t out_dtype; /* R */
+} moe_shape_t;
+
+typedef struct {
+    const float* gamma;  /* [d] RMSNorm scale */
+    const float* W_r;    /* [E][d] router weights, z = v W_r^T */
+    const float* b;      /* [E] selection bias */
+    const void* W_gate;  /* [E][d_ff][d], w_dtype */
+    const void* W_up;    /* [E][d_ff][d], w_dtype */
+    const void* W_down;  /* [E][d][d_ff], w_dtype */
+} moe_weights_t;
+
+/*
+ * Step 1 — RMSNorm [P1 §Norm&Residual, RMSNorm equation]:
+ *   v[t][j] = gamma[j] * x[t][j] / sqrt((1/d) * sum_k x[t][k]^2 + eps)
+ * x [T][d] (x_dt), gamma [d] f32, v [T][d] (v_dt), fp32 arithmetic.
+ * Requires d % 8 == 0; x and v 16-byte aligned.
+ */
+moe_status_t moe_rmsnorm(const void* x, moe_dtype_t x_dt, const float* gamma, int32_t T, int32_t d, float eps,
+                         void* v, moe_dtype_t v_dt, moe_stream_t stream);
+
+/*
+ * Step 2 — router [P1 §专家并行 / MoE Router 过程]:
+ *   z = v W_r^T (fp32),  s = sigmoid(z),  I = TopK(s + b),  w_i = s_i / sum_{j in I} s_j
+ * The bias b only takes part in the choice of I, never in w.  The selection
+ * score is fp32: sigmoid evaluated in double and rounded once, plus b in fp32.
+ * Ties go to the lower expert index; I is written by descending score.
+ * v [T][d] (v_dt), W_r [E][d] f32, b [E] f32.
+ * Outputs: topk_idx [T][k] int32, topk_w [T][k] f32; optional (NULL to skip)
+ * logits [T][E] f32 and margin [T] f32 = k-th score minus the best unpicked
+ * score (+inf when E == k).  Workspace: split-K partial logits.
+ * Requires 1 <= k <= 8, k <= E <= 256, d % 8 == 0.
+ */
+moe_status_t moe_router_topk(const void* v, moe_dtype_t v_dt, const float* W_r, const float* b, int32_t T,
+                             int32_t d, int32_t E, int32_t k, int32_t* topk_idx, float* topk_w, float* logits,
+                             float* margin, void* ws, size_t* ws_bytes, moe_stream_t stream);
+
+/*
+ * Step 3 — token permutation into expert-contiguous rows
+ * [P5 §Token 分发策略, token_permutation; §专家计算实现, contiguous layout]:
+ *   counts[e]      = number of (t, i) with topk_idx[t][i] == e
+ *   offsets[e]     = sum_{e' < e} counts[e'] (no padding), offsets[E] = T*k
+ *   slot_token[r]  = source token of row r (r < T*k)
+ *   token_slot[t][i] = row that holds pick i of token t (-1 if its id was bad)
+ *   xp[r][:]       = v[slot_token[r]][:]   (dtype v_dt)
+ * Rows inside a segment follow ascending token index, so the result is
+ * deterministic.  Bad ids set MOE_DEV_BAD_EXPERT_ID and are dropped.
+ * Requires d % 8 == 0, v and xp 16-byte aligned, 1 <= k <= 8, k <= E <= 256.
+ */
+moe_status_t moe_permute(const void* v, moe_dtype_t v_dt, const int32_t* topk_idx, int32_t T, int32_t d, int32_t E,
+                         int32_t k, int32_t* counts, int32_t* offsets, int32_t* slot_token, int32_t* token_slot,
+                         void* xp, void* ws, size_t* ws_bytes, int32_t* dev_status, moe_stream_t stream);
+
+/*
+ * Step 4, first half — gate/up projections with the SwiGLU product
+ * [P1 §实际 MLP 计算策略: SiLU(X W_gate) ⊙ X W_up; §EP 路径: grouped GEMM]:
+ *   h[r][f] = SiLU(sum_j xp[r][j] W_gate[e][f][j]) * (sum_j xp[r][j] W_up[e][f][j])
+ * for every row r of expert e's segment [offsets[e], offsets[e] + counts[e]).
+ * SiLU(x) = x * sigmoid(x).  dt = MOE_BF16: tcgen05 tensor cores, fp32
+ * accumulation in tensor memory, h rounded to bf16; dt = MOE_F32: fp32 CUDA cores.
+ * xp [S][d], h [S][d_ff] (dtype dt); counts/offsets as written by moe_permute.
+ * Rows outside every segment are not written.
+ * bf16 requires d % 64 == 0, d_ff % 128 == 0, 16-byte aligned pointers.
+ */
+moe_status_t moe_expert_gate_up(const void* xp, const void* W_gate, const void* W_up, moe_dtype_t dt,
+                                const int32_t* counts, const int32_t* offsets, int32_t S, int32_t E, int32_t d,
+                                int32_t d_ff, void* h, int32_t* dev_status, moe_stream_t stream);
+
+/*
+ * Step 4, second half — down projection [P1 §实际 MLP 计算策略, "· W_down"]:
+ *   y[r][o] = sum_f h[r][f] W_down[e][o][f]   for rows r of expert e's segment.
+ * h [S][d_ff], y [S][d] (dtype dt).  bf16 requires d % 128 == 0, d_ff % 64 == 0.
+ */
+moe_status_t moe_expert_down(const void* h, const void* W_down, moe_dtype_t dt, const int32_t* counts,
+                             const int32_t* offsets, int32_t S, int32_t E, int32_t d, int32_t d_ff, void* y,
+                             int32_t* dev_status, moe_stream_t stream);
+
+/*
+ * Step 4 — grouped SwiGLU expert MLP [P1 §实际 MLP 计算策略; §EP 路径;
+ * P5 §专家计算实现, BatchedExperts]: moe_expert_gate_up then moe_expert_down.
+ * h is the caller's [S][d_ff] intermediate.
+ */
+moe_status_t moe_grouped_swiglu(const void* xp, const void* W_gate, const void* W_up, const void* W_down,
+                                moe_dtype_t dt, const int32_t* counts, const int32_t* offsets, int32_t S, int32_t E,
+                                int32_t d, int32_t d_ff, void* h, void* y, int32_t* dev_status, moe_stream_t stream);
+
+/*
+ * Step 5 — weighted un-permute and residual [P1 §EP 路径: weighted sum at the
+ * source; §Norm&Residual: X' = R + FFN(V); P5 token_unpermutation]:
+ *   out[t][j] = residual[t][j] + sum_{i<k} topk_w[t][i] * y[token_slot[t][i]][j]
+ * fp32 accumulation in pick order.  Picks with token_slot == -1 are skipped.
+ * y [T*k][d] (y_dt), residual [T][d] (r_dt), out [T][d] (out_dt).
+ * Requires d % 8 == 0 and 16-byte aligned y, residual, out.
+ */
+moe_status_t moe_unpermute_combine(const void* y, moe_dtype_t y_dt, const int32_t* token_slot, const float* topk_w,
+                                   const void* residual, moe_dtype_t r_dt, int32_t T, int32_t d, int32_t k, void* out,
+                                   moe_dtype_t out_dt, moe_stream_t stream);
+
+/*
+ * The whole layer, steps 1-5 [P1 §Norm&Residual: X_{l+1} = R_l + FFN(RMSNorm(R_l))]:
+ *   out = x + MoE(RMSNorm(x))
+ * The router reads the unrounded fp32 normalised rows; the expert path reads
+ * them rounded to w_dtype.  Optional outputs (NULL to keep them in the
+ * workspace): topk_idx [T][k], topk_w [T][k], logits [T][E].
+ * dev_status is cleared at the start and receives MOE_DEV_* bits.
+ * Supported: x_dtype, out_dtype in {f32, bf16}; w_dtype bf16 (tensor cores,
+ * needs d % 128 == 0, d_ff % 128 == 0) or f32 (CUDA cores, d % 8 == 0,
+ * d_ff % 8 == 0); 1 <= top_k <= 8; top_k <= E <= 256.
+ */
+moe_status_t moe_forward(const moe_shape_t* shape, const moe_weights_t* weights, const void* x, void* out,
+                         int32_t* topk_idx, float* topk_w, float* logits, void* ws, size_t* ws_bytes,
+                         int32_t* dev_status, moe_stream_t stream);
+
+/* Static text for a status code. */
+const char* moe_status_string(moe_status_t status);
+
+/* ABI version of this header (bumped on any incompatible change). */
+#define MOE_ABI_VERSION 1
+int32_t moe_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H */

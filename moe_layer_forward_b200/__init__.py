@@ -1,0 +1,197 @@
+"""MoE layer forward on one B200: Python binding of ``libmoe.so``.
+
+Every function has the name of the C entry point it calls (``include/moe.h``)
+and only marshals torch tensors into pointers, sizes and the current CUDA
+stream.  All arithmetic runs in the library's sm_100a kernels.  Importing the
+package fails loudly if ``libmoe.so`` has not been built.
+
+    R = X + MoE(RMSNorm(X))   (see ``moe_forward``)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m moe_layer_forward_b200.build` "
+                      "(or __graft_entry__.build()); there is no fallback implementation")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+MOE_F32, MOE_BF16 = 0, 1
+MOE_DEV_BAD_EXPERT_ID, MOE_DEV_TIMEOUT = 1, 2
+
+_vp, _i32, _f32, _szp = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.POINTER(ctypes.c_size_t)
+
+
+class MoeShape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("E", ctypes.c_int32), ("top_k", ctypes.c_int32),
+                ("d_ff", ctypes.c_int32), ("eps", ctypes.c_float), ("x_dtype", ctypes.c_int),
+                ("w_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int)]
+
+
+class MoeWeights(ctypes.Structure):
+    _fields_ = [("gamma", _vp), ("W_r", _vp), ("b", _vp), ("W_gate", _vp), ("W_up", _vp), ("W_down", _vp)]
+
+
+_sig = {
+    "moe_rmsnorm": [_vp, _i32, _vp, _i32, _i32, _f32, _vp, _i32, _vp],
+    "moe_router_topk": [_vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _szp, _vp],
+    "moe_permute": [_vp, _i32, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _szp, _vp, _vp],
+    "moe_expert_gate_up": [_vp, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp],
+    "moe_expert_down": [_vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp],
+    "moe_grouped_swiglu": [_vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp],
+    "moe_unpermute_combine": [_vp, _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _i32, _vp],
+    "moe_forward": [ctypes.POINTER(MoeShape), ctypes.POINTER(MoeWeights), _vp, _vp, _vp, _vp, _vp, _vp, _szp, _vp,
+                    _vp],
+}
+for _name, _args in _sig.items():
+    _fn = getattr(_lib, _name)
+    _fn.argtypes = _args
+    _fn.restype = ctypes.c_int
+_lib.moe_status_string.argtypes = [ctypes.c_int]
+_lib.moe_status_string.restype = ctypes.c_char_p
+_lib.moe_abi_version.restype = ctypes.c_int32
+
+
+class MoEError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn}: {_lib.moe_status_string(status).decode()} (status {status})")
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        raise MoEError(fn, status)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return MOE_F32
+    if t.dtype == torch.bfloat16:
+        return MOE_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _p(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors passed to libmoe must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libmoe must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(dev=None):
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _ws(query, device) -> torch.Tensor:
+    n = ctypes.c_size_t(0)
+    query(None, ctypes.byref(n))
+    return torch.empty(max(int(n.value), 1), dtype=torch.uint8, device=device)
+
+
+def abi_version() -> int:
+    return int(_lib.moe_abi_version())
+
+
+def moe_rmsnorm(x: torch.Tensor, gamma: torch.Tensor, eps: float, v: torch.Tensor) -> None:
+    T, d = x.shape
+    _check("moe_rmsnorm", _lib.moe_rmsnorm(_p(x), _dt(x), _p(gamma), T, d, eps, _p(v), _dt(v), _stream(x.device)))
+
+
+def moe_router_topk(v, W_r, b, topk_idx, topk_w, logits=None, margin=None, ws=None) -> None:
+    T, d = v.shape
+    E = W_r.shape[0]
+    k = topk_idx.shape[1]
+
+    def call(wsp, nbytes):
+        return _lib.moe_router_topk(_p(v), _dt(v), _p(W_r), _p(b), T, d, E, k, _p(topk_idx), _p(topk_w), _p(logits),
+                                    _p(margin), wsp, nbytes, _stream(v.device))
+
+    if ws is None:
+        ws = _ws(lambda w, n: _check("moe_router_topk", call(w, n)), v.device)
+    n = ctypes.c_size_t(ws.numel())
+    _check("moe_router_topk", call(_p(ws), ctypes.byref(n)))
+
+
+def moe_permute(v, topk_idx, E: int, counts, offsets, slot_token, token_slot, xp, ws=None, dev_status=None) -> None:
+    T, d = v.shape
+    k = topk_idx.shape[1]
+
+    def call(wsp, nbytes):
+        return _lib.moe_permute(_p(v), _dt(v), _p(topk_idx), T, d, E, k, _p(counts), _p(offsets), _p(slot_token),
+                                _p(token_slot), _p(xp), wsp, nbytes, _p(dev_status), _stream(v.device))
+
+    if ws is None:
+        ws = _ws(lambda w, n: _check("moe_permute", call(w, n)), v.device)
+    n = ctypes.c_size_t(ws.numel())
+    _check("moe_permute", call(_p(ws), ctypes.byref(n)))
+
+
+def moe_expert_gate_up(xp, W_gate, W_up, counts, offsets, h, dev_status=None) -> None:
+    S, d = xp.shape
+    E, d_ff, _ = W_gate.shape
+    _check("moe_expert_gate_up", _lib.moe_expert_gate_up(_p(xp), _p(W_gate), _p(W_up), _dt(W_gate), _p(counts),
+                                                         _p(offsets), S, E, d, d_ff, _p(h), _p(dev_status),
+                                                         _stream(xp.device)))
+
+
+def moe_expert_down(h, W_down, counts, offsets, y, dev_status=None) -> None:
+    S, d_ff = h.shape
+    E, d, _ = W_down.shape
+    _check("moe_expert_down", _lib.moe_expert_down(_p(h), _p(W_down), _dt(W_down), _p(counts), _p(offsets), S, E, d,
+                                                   d_ff, _p(y), _p(dev_status), _stream(h.device)))
+
+
+def moe_grouped_swiglu(xp, W_gate, W_up, W_down, counts, offsets, h, y, dev_status=None) -> None:
+    S, d = xp.shape
+    E, d_ff, _ = W_gate.shape
+    _check("moe_grouped_swiglu", _lib.moe_grouped_swiglu(_p(xp), _p(W_gate), _p(W_up), _p(W_down), _dt(W_gate),
+                                                         _p(counts), _p(offsets), S, E, d, d_ff, _p(h), _p(y),
+                                                         _p(dev_status), _stream(xp.device)))
+
+
+def moe_unpermute_combine(y, token_slot, topk_w, residual, out) -> None:
+    T, d = residual.shape
+    k = token_slot.shape[1]
+    _check("moe_unpermute_combine", _lib.moe_unpermute_combine(_p(y), _dt(y), _p(token_slot), _p(topk_w),
+                                                               _p(residual), _dt(residual), T, d, k, _p(out),
+                                                               _dt(out), _stream(residual.device)))
+
+
+def _shape(x, W_gate, out, top_k, eps, E) -> MoeShape:
+    T, d = x.shape
+    _, d_ff, _ = W_gate.shape
+    return MoeShape(T, d, E, top_k, d_ff, eps, _dt(x), _dt(W_gate), _dt(out))
+
+
+def forward_workspace_bytes(x, W_r, W_gate, out, top_k: int = 8, eps: float = 1e-5) -> int:
+    """Bytes of workspace ``moe_forward`` needs for these tensors (device query; queues nothing)."""
+    shp = _shape(x, W_gate, out, top_k, eps, W_r.shape[0])
+    wts = MoeWeights()
+    n = ctypes.c_size_t(0)
+    _check("moe_forward", _lib.moe_forward(ctypes.byref(shp), ctypes.byref(wts), None, None, None, None, None, None,
+                                           ctypes.byref(n), None, _stream(x.device)))
+    return int(n.value)
+
+
+def moe_forward(x, gamma, W_r, b, W_gate, W_up, W_down, out, top_k: int = 8, eps: float = 1e-5, topk_idx=None,
+                topk_w=None, logits=None, ws=None, dev_status=None) -> None:
+    """out = x + MoE(RMSNorm(x)) on x's device and current stream (asynchronous)."""
+    shp = _shape(x, W_gate, out, top_k, eps, W_r.shape[0])
+    wts = MoeWeights(_p(gamma), _p(W_r), _p(b), _p(W_gate), _p(W_up), _p(W_down))
+    if ws is None:
+        ws = torch.empty(max(forward_workspace_bytes(x, W_r, W_gate, out, top_k, eps), 1), dtype=torch.uint8,
+                         device=x.device)
+    n = ctypes.c_size_t(ws.numel())
+    _check("moe_forward", _lib.moe_forward(ctypes.byref(shp), ctypes.byref(wts), _p(x), _p(out), _p(topk_idx),
+                                           _p(topk_w), _p(logits), _p(ws), ctypes.byref(n), _p(dev_status),
+                                           _stream(x.device)))

@@ -1,0 +1,327 @@
+// C ABI of libmoe.so (declared in include/moe.h): argument checks, workspace
+// layout and the launch sequence of the MoE layer forward.  No entry point
+// allocates, synchronises with the host, throws or aborts.
+#include <stdint.h>
+#include <string.h>
+
+#include "kernels.h"
+#include "moe.h"
+
+using namespace moe;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DevCache {
+    int sms = 0;
+    int major = 0;
+};
+DevCache g_dev[kMaxDevices];
+
+moe_status_t make_ctx(moe_stream_t stream, Ctx& c) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_DEVICE;
+    DevCache& dc = g_dev[dev];
+    if (dc.sms == 0) {
+        int sms = 0, major = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return MOE_ERR_CUDA;
+        }
+        dc.major = major;
+        dc.sms = sms;
+    }
+    if (dc.major != 10) return MOE_ERR_DEVICE;
+    c.stream = reinterpret_cast<cudaStream_t>(stream);
+    c.num_sms = dc.sms;
+    c.device = dev;
+    return MOE_OK;
+}
+
+moe_status_t cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return MOE_OK;
+    cudaGetLastError();  // clear the non-sticky error so the caller's next call is not affected
+    return MOE_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool valid_dt(moe_dtype_t t) { return t == MOE_F32 || t == MOE_BF16; }
+size_t esize(moe_dtype_t t) { return t == MOE_BF16 ? 2 : 4; }
+
+// bump allocator over the caller's workspace; with base == nullptr it only measures
+struct Carve {
+    uint8_t* base;
+    size_t off = 0;
+    explicit Carve(void* b) : base(static_cast<uint8_t*>(b)) {}
+    void* take(size_t bytes) {
+        const size_t o = (off + 255) & ~size_t(255);
+        off = o + bytes;
+        return base ? base + o : nullptr;
+    }
+};
+
+moe_status_t check_ws(void* ws, size_t* ws_bytes, size_t need, bool* query_only) {
+    *query_only = false;
+    if (!ws_bytes) return MOE_ERR_INVALID_ARG;
+    if (!ws) {
+        *ws_bytes = need;
+        *query_only = true;
+        return MOE_OK;
+    }
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_INVALID_ARG;
+    if (*ws_bytes < need) {
+        *ws_bytes = need;
+        return MOE_ERR_WORKSPACE;
+    }
+    return MOE_OK;
+}
+
+moe_status_t check_router_shape(int T, int d, int E, int k) {
+    if (T < 0 || d <= 0 || E <= 0 || k <= 0) return MOE_ERR_INVALID_ARG;
+    if (k > MOE_MAX_TOP_K || E > MOE_MAX_EXPERTS || k > E) return MOE_ERR_UNSUPPORTED;
+    if (d % 8 != 0) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+moe_status_t check_expert_shape(moe_dtype_t dt, int S, int E, int d, int d_ff) {
+    if (S < 0 || E <= 0 || d <= 0 || d_ff <= 0) return MOE_ERR_INVALID_ARG;
+    if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+    if (dt == MOE_BF16) {
+        if (d % 128 != 0 || d_ff % 128 != 0) return MOE_ERR_UNSUPPORTED;
+    } else if (dt == MOE_F32) {
+        if (d % 8 != 0 || d_ff % 8 != 0) return MOE_ERR_UNSUPPORTED;
+    } else {
+        return MOE_ERR_INVALID_ARG;
+    }
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status_t s) {
+    switch (s) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+        case MOE_ERR_WORKSPACE: return "workspace too small";
+        case MOE_ERR_CUDA: return "CUDA error";
+        case MOE_ERR_DEVICE: return "device is not sm_100";
+    }
+    return "unknown status";
+}
+
+int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+moe_status_t moe_rmsnorm(const void* x, moe_dtype_t x_dt, const float* gamma, int32_t T, int32_t d, float eps,
+                         void* v, moe_dtype_t v_dt, moe_stream_t stream) {
+    if (T < 0 || d <= 0 || !valid_dt(x_dt) || !valid_dt(v_dt)) return MOE_ERR_INVALID_ARG;
+    if (d % 8 != 0) return MOE_ERR_UNSUPPORTED;
+    if (T == 0) return MOE_OK;
+    if (!x || !gamma || !v || !aligned16(x) || !aligned16(v) || !aligned16(gamma)) return MOE_ERR_INVALID_ARG;
+    Ctx c;
+    moe_status_t st = make_ctx(stream, c);
+    if (st != MOE_OK) return st;
+    return cuda_status(launch_rmsnorm(c, x, x_dt, gamma, T, d, eps, v, v_dt, nullptr));
+}
+
+moe_status_t moe_router_topk(const void* v, moe_dtype_t v_dt, const float* W_r, const float* b, int32_t T,
+                             int32_t d, int32_t E, int32_t k, int32_t* topk_idx, float* topk_w, float* logits,
+                             float* margin, void* ws, size_t* ws_bytes, moe_stream_t stream) {
+    moe_status_t st = check_router_shape(T, d, E, k);
+    if (st != MOE_OK) return st;
+    if (!valid_dt(v_dt)) return MOE_ERR_INVALID_ARG;
+    Ctx c;
+    st = make_ctx(stream, c);
+    if (st != MOE_OK) return st;
+    const RouterPlan plan = plan_router(T, d, E, c.num_sms);
+    Carve cv(nullptr);
+    cv.take(plan.partial_bytes);
+    bool query = false;
+    st = check_ws(ws, ws_bytes, cv.off, &query);
+    if (st != MOE_OK || query || T == 0) return st;
+    if (!v || !W_r || !b || !topk_idx || !topk_w || !aligned16(v) || !aligned16(W_r)) return MOE_ERR_INVALID_ARG;
+    Carve w(ws);
+    float* partial = static_cast<float*>(w.take(plan.partial_bytes));
+    st = cuda_status(launch_router_logits(c, plan, v, v_dt, nullptr, nullptr, W_r, T, d, E, partial));
+    if (st != MOE_OK) return st;
+    return cuda_status(launch_router_topk(c, plan, partial, b, T, E, k, topk_idx, topk_w, logits, margin));
+}
+
+moe_status_t moe_permute(const void* v, moe_dtype_t v_dt, const int32_t* topk_idx, int32_t T, int32_t d, int32_t E,
+                         int32_t k, int32_t* counts, int32_t* offsets, int32_t* slot_token, int32_t* token_slot,
+                         void* xp, void* ws, size_t* ws_bytes, int32_t* dev_status, moe_stream_t stream) {
+    moe_status_t st = check_router_shape(T, d, E, k);
+    if (st != MOE_OK) return st;
+    if (!valid_dt(v_dt)) return MOE_ERR_INVALID_ARG;
+    Carve cv(nullptr);
+    cv.take(permute_ws_bytes(T, E));
+    bool query = false;
+    st = check_ws(ws, ws_bytes, cv.off, &query);
+    if (st != MOE_OK || query) return st;
+    if (!counts || !offsets) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!v || !topk_idx || !slot_token || !token_slot || !xp || !aligned16(v) || !aligned16(xp)))
+        return MOE_ERR_INVALID_ARG;
+    Ctx c;
+    st = make_ctx(stream, c);
+    if (st != MOE_OK) return st;
+    Carve w(ws);
+    int32_t* hist = static_cast<int32_t*>(w.take(permute_ws_bytes(T, E)));
+    return cuda_status(launch_permute(c, v, v_dt, topk_idx, T, d, E, k, counts, offsets, slot_token, token_slot, xp,
+                                      hist, dev_status));
+}
+
+moe_status_t moe_expert_gate_up(const void* xp, const void* W_gate, const void* W_up, moe_dtype_t dt,
+                                const int32_t* counts, const int32_t* offsets, int32_t S, int32_t E, int32_t d,
+                                int32_t d_ff, void* h, int32_t* dev_status, moe_stream_t stream) {
+    moe_status_t st = check_expert_shape(dt, S, E, d, d_ff);
+    if (st != MOE_OK) return st;
+    if (S == 0) return MOE_OK;
+    if (!xp || !W_gate || !W_up || !counts || !offsets || !h) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(xp) || !aligned16(W_gate) || !aligned16(W_up) || !aligned16(h)) return MOE_ERR_INVALID_ARG;
+    Ctx c;
+    st = make_ctx(stream, c);
+    if (st != MOE_OK) return st;
+    if (dt == MOE_BF16)
+        return cuda_status(launch_gate_up_bf16(c, xp, W_gate, W_up, counts, offsets, S, E, d, d_ff, h, dev_status));
+    return cuda_status(launch_gate_up_f32(c, static_cast<const float*>(xp), static_cast<const float*>(W_gate),
+                                          static_cast<const float*>(W_up), counts, offsets, S, E, d, d_ff,
+                                          static_cast<float*>(h)));
+}
+
+moe_status_t moe_expert_down(const void* h, const void* W_down, moe_dtype_t dt, const int32_t* counts,
+                             const int32_t* offsets, int32_t S, int32_t E, int32_t d, int32_t d_ff, void* y,
+                             int32_t* dev_status, moe_stream_t stream) {
+    moe_status_t st = check_expert_shape(dt, S, E, d, d_ff);
+    if (st != MOE_OK) return st;
+    if (S == 0) return MOE_OK;
+    if (!h || !W_down || !counts || !offsets || !y) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(h) || !aligned16(W_down) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+    Ctx c;
+    st = make_ctx(stream, c);
+    if (st != MOE_OK) return st;
+    if (dt == MOE_BF16) return cuda_status(launch_down_bf16(c, h, W_down, counts, offsets, S, E, d, d_ff, y, dev_status));
+    return cuda_status(launch_down_f32(c, static_cast<const float*>(h), static_cast<const float*>(W_down), counts,
+                                       offsets, S, E, d, d_ff, static_cast<float*>(y)));
+}
+
+moe_status_t moe_grouped_swiglu(const void* xp, const void* W_gate, const void* W_up, const void* W_down,
+                                moe_dtype_t dt, const int32_t* counts, const int32_t* offsets, int32_t S, int32_t E,
+                                int32_t d, int32_t d_ff, void* h, void* y, int32_t* dev_status, moe_stream_t stream) {
+    moe_status_t st = check_expert_shape(dt, S, E, d, d_ff);
+    if (st != MOE_OK) return st;
+    if (S > 0 && !W_down) return MOE_ERR_INVALID_ARG;
+    st = moe_expert_gate_up(xp, W_gate, W_up, dt, counts, offsets, S, E, d, d_ff, h, dev_status, stream);
+    if (st != MOE_OK) return st;
+    return moe_expert_down(h, W_down, dt, counts, offsets, S, E, d, d_ff, y, dev_status, stream);
+}
+
+moe_status_t moe_unpermute_combine(const void* y, moe_dtype_t y_dt, const int32_t* token_slot, const float* topk_w,
+                                   const void* residual, moe_dtype_t r_dt, int32_t T, int32_t d, int32_t k, void* out,
+                                   moe_dtype_t out_dt, moe_stream_t stream) {
+    if (T < 0 || d <= 0 || k <= 0 || !valid_dt(y_dt) || !valid_dt(r_dt) || !valid_dt(out_dt))
+        return MOE_ERR_INVALID_ARG;
+    if (k > MOE_MAX_TOP_K || d % 8 != 0) return MOE_ERR_UNSUPPORTED;
+    if (T == 0) return MOE_OK;
+    if (!y || !token_slot || !topk_w || !residual || !out) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(y) || !aligned16(residual) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+    Ctx c;
+    moe_status_t st = make_ctx(stream, c);
+    if (st != MOE_OK) return st;
+    return cuda_status(launch_combine(c, y, y_dt, token_slot, topk_w, residual, r_dt, T, d, k, out, out_dt));
+}
+
+moe_status_t moe_forward(const moe_shape_t* shape, const moe_weights_t* wts, const void* x, void* out,
+                         int32_t* topk_idx, float* topk_w, float* logits, void* ws, size_t* ws_bytes,
+                         int32_t* dev_status, moe_stream_t stream) {
+    if (!shape || !wts || !ws_bytes) return MOE_ERR_INVALID_ARG;
+    const int T = shape->T, d = shape->d, E = shape->E, k = shape->top_k, d_ff = shape->d_ff;
+    if (!valid_dt(shape->x_dtype) || !valid_dt(shape->w_dtype) || !valid_dt(shape->out_dtype))
+        return MOE_ERR_INVALID_ARG;
+    moe_status_t st = check_router_shape(T, d, E, k);
+    if (st != MOE_OK) return st;
+    const moe_dtype_t wdt = shape->w_dtype;
+    if ((int64_t)T * k > INT32_MAX / 2) return MOE_ERR_UNSUPPORTED;
+    const int S = T * k;
+    st = check_expert_shape(wdt, S, E, d, d_ff);
+    if (st != MOE_OK) return st;
+    Ctx c;
+    st = make_ctx(stream, c);
+    if (st != MOE_OK) return st;
+    const RouterPlan plan = plan_router(T, d, E, c.num_sms);
+    const size_t es = esize(wdt);
+
+    // workspace layout (each piece 256-byte aligned)
+    Carve cv(ws);
+    void* v = cv.take((size_t)T * d * es);
+    float* rstd = static_cast<float*>(cv.take((size_t)T * sizeof(float)));
+    float* partial = static_cast<float*>(cv.take(plan.partial_bytes));
+    // routing is kept in the workspace unless the caller asks for it (the size never depends on that)
+    int32_t* idx_ws = static_cast<int32_t*>(cv.take((size_t)S * sizeof(int32_t)));
+    float* wgt_ws = static_cast<float*>(cv.take((size_t)S * sizeof(float)));
+    int32_t* idx = topk_idx ? topk_idx : idx_ws;
+    float* wgt = topk_w ? topk_w : wgt_ws;
+    int32_t* hist = static_cast<int32_t*>(cv.take(permute_ws_bytes(T, E)));
+    int32_t* counts = static_cast<int32_t*>(cv.take((size_t)E * sizeof(int32_t)));
+    int32_t* offsets = static_cast<int32_t*>(cv.take((size_t)(E + 1) * sizeof(int32_t)));
+    int32_t* slot_token = static_cast<int32_t*>(cv.take((size_t)S * sizeof(int32_t)));
+    int32_t* token_slot = static_cast<int32_t*>(cv.take((size_t)S * sizeof(int32_t)));
+    void* xp = cv.take((size_t)S * d * es);
+    void* h = cv.take((size_t)S * d_ff * es);
+    void* y = cv.take((size_t)S * d * es);
+    bool query = false;
+    st = check_ws(ws, ws_bytes, cv.off, &query);
+    if (st != MOE_OK || query) return st;
+
+    const bool need_w = T > 0;
+    if (need_w && (!x || !out || !wts->gamma || !wts->W_r || !wts->b || !wts->W_gate || !wts->W_up || !wts->W_down))
+        return MOE_ERR_INVALID_ARG;
+    if (need_w && (!aligned16(x) || !aligned16(out) || !aligned16(wts->gamma) || !aligned16(wts->W_r) ||
+                   !aligned16(wts->W_gate) || !aligned16(wts->W_up) || !aligned16(wts->W_down)))
+        return MOE_ERR_INVALID_ARG;
+
+    if (dev_status) {
+        st = cuda_status(cudaMemsetAsync(dev_status, 0, sizeof(int32_t), c.stream));
+        if (st != MOE_OK) return st;
+    }
+    if (T == 0) return MOE_OK;
+    const int xdt = shape->x_dtype;
+    // 1. RMSNorm: v rounded to the expert dtype, and 1/rms for the router
+    st = cuda_status(launch_rmsnorm(c, x, xdt, wts->gamma, T, d, shape->eps, v, wdt, rstd));
+    if (st != MOE_OK) return st;
+    // 2. router on the unrounded fp32 normalised rows (x * rstd * gamma formed in the GEMM)
+    st = cuda_status(launch_router_logits(c, plan, x, xdt, rstd, wts->gamma, wts->W_r, T, d, E, partial));
+    if (st != MOE_OK) return st;
+    st = cuda_status(launch_router_topk(c, plan, partial, wts->b, T, E, k, idx, wgt, logits, nullptr));
+    if (st != MOE_OK) return st;
+    // 3. permutation
+    st = cuda_status(launch_permute(c, v, wdt, idx, T, d, E, k, counts, offsets, slot_token, token_slot, xp, hist,
+                                    dev_status));
+    if (st != MOE_OK) return st;
+    // 4. grouped SwiGLU MLP
+    if (wdt == MOE_BF16) {
+        st = cuda_status(launch_gate_up_bf16(c, xp, wts->W_gate, wts->W_up, counts, offsets, S, E, d, d_ff, h,
+                                             dev_status));
+        if (st != MOE_OK) return st;
+        st = cuda_status(launch_down_bf16(c, h, wts->W_down, counts, offsets, S, E, d, d_ff, y, dev_status));
+    } else {
+        st = cuda_status(launch_gate_up_f32(c, static_cast<const float*>(xp), static_cast<const float*>(wts->W_gate),
+                                            static_cast<const float*>(wts->W_up), counts, offsets, S, E, d, d_ff,
+                                            static_cast<float*>(h)));
+        if (st != MOE_OK) return st;
+        st = cuda_status(launch_down_f32(c, static_cast<const float*>(h), static_cast<const float*>(wts->W_down),
+                                         counts, offsets, S, E, d, d_ff, static_cast<float*>(y)));
+    }
+    if (st != MOE_OK) return st;
+    // 5. weighted un-permute + residual
+    return cuda_status(launch_combine(c, y, wdt, token_slot, wgt, x, xdt, T, d, k, out, shape->out_dtype));
+}
+
+}  // extern "C"

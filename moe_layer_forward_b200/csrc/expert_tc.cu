@@ -1,0 +1,624 @@
+// Step 4 for bf16 expert weights: grouped GEMMs on the 5th-generation tensor
+// cores (tcgen05.mma, accumulators in tensor memory, operands staged by TMA).
+//
+// "推理计算流梳理" (huanyp.cn), §实际 MLP 计算策略: Y = (SiLU(X W_gate) ⊙ X W_up) W_down;
+// §EP 路径: the active experts of a rank run as one grouped GEMM.  The Chitu MoE
+// page (§专家计算实现) describes the prefill layout this kernel consumes: the rows
+// of each expert are contiguous ("deepgemm_contiguous"); its FP8/Hopper kernels
+// are prior art, not the design here.
+//
+// One persistent kernel template covers both halves of the expert MLP:
+//   gate/up: h = SiLU(xp W_gate^T) ⊙ (xp W_up^T)   (SwiGLU fused in the epilogue)
+//   down:    y = h W_down^T
+// A work tile is (expert e, row block rb, column block cb).  Tiles are
+// numbered expert-major, then column block, then row block, and CTAs take
+// tiles tile = blockIdx.x + i * gridDim.x, so the row blocks that share a
+// weight tile run side by side and read it from L2 once.  The per-expert row
+// counts live only on the device; every CTA turns them into a tile prefix
+// sum in shared memory (no host sync).
+//
+// Two operand arrangements:
+//   rows-as-M (prefill, many rows per expert): MMA M = 128 activation rows,
+//     N = 256 weight rows (gate|up stacked, or 256 down rows).
+//   weights-as-M (decode, few rows per expert): MMA M = 128 weight rows,
+//     N = the expert's row count rounded up to 16 (<= R), so an expert with
+//     8 tokens costs an N=16 MMA rather than a 128-row one.  The kernel then
+//     streams weights and is bound by HBM.
+//
+// Warp roles (192 threads, 1 CTA per SM):
+//   warp 0      TMA producer: a STAGES-deep ring of 64-wide K slices (128-byte
+//               swizzled rows), one mbarrier pair (full/empty) per stage.
+//   warp 1      owns the tensor-memory allocation; lane 0 issues tcgen05.mma
+//               (4 x K=16 per stage) and tcgen05.commit to release each stage
+//               and to publish a finished accumulator.
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator (each warp its 32 TMEM
+//               lanes), SiLU(g)*u in fp32, bf16 stores.  Two accumulator
+//               buffers let the epilogue of one tile overlap the next tile's MMAs.
+// Every wait is bounded (globaltimer); a wait that gives up raises
+// DEV_TIMEOUT in the status word and all roles unwind, drain in-flight copies
+// and MMAs, free tensor memory and exit.
+#include <cuda.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace tc {
+
+constexpr int BK = 64;  // K elements per stage = one 128-byte swizzle row of bf16
+constexpr int kThreads = 192;
+constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s per wait
+constexpr int kSmemLimit = 232448;              // 227 KB opt-in per CTA
+
+// ----------------------------------------------------------------------------- PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Wait for the phase of the given parity to complete.  Gives up after
+// kTimeoutNs, or early once another role has raised the abort flag.
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 127u) == 0u) {
+            if (*abort_flag) return false;
+            if (globaltimer() - t0 > kTimeoutNs) return false;
+        }
+    }
+}
+
+// Every lane of the warp waits; the result is the same for all lanes.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    const bool ok = mbar_wait(bar, parity, abort_flag);
+    return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ void tma_prefetch(const CUtensorMap* tm) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tm)) : "memory");
+}
+// 2-D tiled TMA load (box set in the tensor map) into shared memory; completion
+// is counted in bytes on the mbarrier.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* tm, int x, int y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            dst),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t slot, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot), "r"(ncols) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+// arrive on the mbarrier once all tcgen05 operations issued so far by this thread are complete
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+// D[tmem] (+)= A[smem] * B[smem]^T, both K-major; accumulate when acc != 0
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
+// 32 TMEM lanes (this warp's quarter) x 32 consecutive 32-bit columns; thread i gets lane base+i.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+// Wait for this thread's tcgen05.ld results.  The registers are passed through
+// so that no use of them can be scheduled before the wait.
+template <int N>
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[N]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+template <int N>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[N]) {
+    if constexpr (N == 32) tmem_ld32(taddr, r);
+    else tmem_ld16(taddr, r);
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
+// 128 B, 8-row groups 1024 B apart (SBO), descriptor version 1 (sm_100).
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// Instruction descriptor, kind::f16: D f32, A and B bf16, both K-major, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+
+// ----------------------------------------------------------------------------- configuration
+template <bool SWAP, bool SWIGLU, int R, int COLS>
+struct Cfg {
+    // SWAP = weights are the MMA's A operand (M = 128 weight rows), activations B (N <= R).
+    static_assert(!SWAP || COLS == 128, "weights-as-M tiles cover 128 weight rows");
+    static_assert(SWAP || R == 128, "rows-as-M tiles cover 128 activation rows");
+    static_assert(R % 16 == 0 && R >= 16 && R <= 256, "row block");
+    static constexpr int MMA_N = SWAP ? R : (SWIGLU ? 2 * COLS : COLS);
+    static_assert(MMA_N % 16 == 0 && MMA_N <= 256, "MMA N for M = 128");
+    static constexpr int A_ROWS = SWAP ? 128 : R;
+    static constexpr int NUM_A = (SWAP && SWIGLU) ? 2 : 1;
+    static constexpr int B_ROWS = SWAP ? R : MMA_N;
+    static constexpr int A_BYTES = A_ROWS * 128;
+    static constexpr int B_BYTES = B_ROWS * 128;
+    static constexpr int STAGE_BYTES = NUM_A * A_BYTES + B_BYTES;
+    static constexpr int WBOX = SWAP ? 128 : (SWIGLU ? 128 : COLS);  // weight rows per TMA box
+    // accumulator columns per buffer: SWAP+SWIGLU keeps gate and up side by side
+    static constexpr int ACC = SWAP ? (SWIGLU ? 2 * R : R) : MMA_N;
+    static constexpr int TMEM_COLS = (2 * ACC <= 32) ? 32 : (2 * ACC <= 64) ? 64 : (2 * ACC <= 128) ? 128 : (2 * ACC <= 256) ? 256 : 512;
+    static_assert(2 * ACC <= 512, "two accumulator buffers must fit in 512 TMEM columns");
+    static constexpr int AUX_BYTES = 4096;  // barriers, tile tables
+    static constexpr int STAGES_MAX = (kSmemLimit - 1024 - AUX_BYTES) / STAGE_BYTES;
+    static constexpr int STAGES = STAGES_MAX > 12 ? 12 : STAGES_MAX;
+    static_assert(STAGES >= 2, "pipeline depth");
+    static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + AUX_BYTES;
+    static constexpr int LDW = R < 32 ? R : 32;  // TMEM columns per tcgen05.ld in the weights-as-M epilogue
+};
+
+struct Args {
+    const int32_t* counts;
+    const int32_t* offsets;
+    int E;
+    int K;      // reduction length (d for gate/up, d_ff for down)
+    int n_out;  // weight rows per expert = output columns
+    uint16_t* out;
+    int64_t ldo;
+    int32_t* status;
+};
+
+struct Aux {  // lives after the stage ring in shared memory
+    uint64_t full[12];
+    uint64_t empty[12];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint64_t drain;
+    uint32_t tmem_slot;
+    int abort_flag;
+    int tstart[kMaxExperts + 1];
+    int cnt[kMaxExperts];
+    int off[kMaxExperts];
+};
+
+__device__ __forceinline__ void decode_tile(const Aux& a, int E, int R, int tile, int& e, int& rb, int& cb) {
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (a.tstart[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    e = lo;
+    const int local = tile - a.tstart[e];
+    const int nrb = (a.cnt[e] + R - 1) / R;
+    cb = local / nrb;
+    rb = local - cb * nrb;
+}
+
+template <bool SWAP, bool SWIGLU, int R, int COLS>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_w1,
+                        const __grid_constant__ CUtensorMap tm_w2, const Args p) {
+    using C = Cfg<SWAP, SWIGLU, R, COLS>;
+    constexpr int STAGES = C::STAGES;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Aux& aux = *reinterpret_cast<Aux*>(smem + STAGES * C::STAGE_BYTES);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    volatile int* abort_flag = &aux.abort_flag;
+
+    // ---- prologue (overlaps the previous kernel's tail under PDL)
+    if (warp == 0 && lane == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_u32(&aux.full[s]), 1);
+            mbar_init(smem_u32(&aux.empty[s]), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&aux.tfull[b]), 1);
+            mbar_init(smem_u32(&aux.tempty[b]), 4);
+        }
+        mbar_init(smem_u32(&aux.drain), 1);
+        aux.abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch(&tm_act);
+        tma_prefetch(&tm_w1);
+        if (SWIGLU) tma_prefetch(&tm_w2);
+    }
+    if (warp == 1) tmem_alloc(smem_u32(&aux.tmem_slot), C::TMEM_COLS);
+
+    pdl_wait();
+    const int E = p.E;
+    for (int e = threadIdx.x; e < E; e += kThreads) {
+        aux.cnt[e] = p.counts[e];
+        aux.off[e] = p.offsets[e];
+    }
+    __syncthreads();
+    if (warp == 0) {
+        // tile prefix over experts: lane owns experts 8*lane .. 8*lane+7
+        const int ncb = p.n_out / COLS;
+        int loc[8], sum = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int e = lane * 8 + i;
+            loc[i] = (e < E) ? ((aux.cnt[e] + R - 1) / R) * ncb : 0;
+            sum += loc[i];
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += n;
+        }
+        int run = incl - sum;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int e = lane * 8 + i;
+            if (e < E) aux.tstart[e] = run;
+            run += loc[i];
+        }
+        if (lane == 31) aux.tstart[E] = incl;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    pdl_trigger();
+    const uint32_t tmem_base = aux.tmem_slot;
+    const int total = aux.tstart[E];
+
+    if (warp == 0) {
+        // ================= TMA producer
+        int stage = 0;
+        uint32_t phase = 0;
+        uint32_t used = 0, last_parity = 0;
+        const int nk = p.K / BK;
+        for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+            int e, rb, cb;
+            decode_tile(aux, E, R, tile, e, rb, cb);
+            const int act_row = aux.off[e] + rb * R;
+            const int w_row = e * p.n_out + cb * COLS;
+            for (int kb = 0; kb < nk; ++kb) {
+                const uint32_t full = smem_u32(&aux.full[stage]), empty = smem_u32(&aux.empty[stage]);
+                if (!warp_wait(empty, phase ^ 1u, abort_flag)) {
+                    if (lane == 0) {
+                        *abort_flag = 1;
+                        set_status(p.status, DEV_TIMEOUT);
+                    }
+                    break;
+                }
+                if (lane == 0) {
+                    uint8_t* st = smem + stage * C::STAGE_BYTES;
+                    const uint32_t a0 = smem_u32(st);
+                    mbar_expect_tx(full, C::STAGE_BYTES);
+                    if constexpr (!SWAP) {
+                        tma_load_2d(a0, &tm_act, kb * BK, act_row, full);
+                        tma_load_2d(a0 + C::A_BYTES, &tm_w1, kb * BK, w_row, full);
+                        if (SWIGLU) tma_load_2d(a0 + C::A_BYTES + 128 * 128, &tm_w2, kb * BK, w_row, full);
+                    } else {
+                        tma_load_2d(a0, &tm_w1, kb * BK, w_row, full);
+                        if (SWIGLU) tma_load_2d(a0 + C::A_BYTES, &tm_w2, kb * BK, w_row, full);
+                        tma_load_2d(a0 + C::NUM_A * C::A_BYTES, &tm_act, kb * BK, act_row, full);
+                    }
+                }
+                used |= 1u << stage;
+                last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        // make sure no copy into this CTA's shared memory is still in flight
+        for (int s = 0; s < STAGES; ++s)
+            if (used & (1u << s)) mbar_wait(smem_u32(&aux.full[s]), (last_parity >> s) & 1u, abort_flag);
+    } else if (warp == 1) {
+        // ================= MMA issuer
+        int stage = 0;
+        uint32_t phase = 0;
+        const int nk = p.K / BK;
+        int j = 0;
+        for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x, ++j) {
+            const int buf = j & 1;
+            const uint32_t use = (uint32_t)(j >> 1);
+            if (!warp_wait(smem_u32(&aux.tempty[buf]), (use & 1u) ^ 1u, abort_flag)) {
+                if (lane == 0) {
+                    *abort_flag = 1;
+                    set_status(p.status, DEV_TIMEOUT);
+                }
+                break;
+            }
+            tc_fence_after();
+            uint32_t idesc;
+            if constexpr (SWAP) {
+                int e, rb, cb;
+                decode_tile(aux, E, R, tile, e, rb, cb);
+                const int rows = min(R, aux.cnt[e] - rb * R);
+                idesc = idesc_bf16(128, (rows + 15) & ~15);
+            } else {
+                idesc = idesc_bf16(128, C::MMA_N);
+            }
+            const uint32_t d_tmem = tmem_base + (uint32_t)(buf * C::ACC);
+            bool ok = true;
+            for (int kb = 0; kb < nk; ++kb) {
+                if (!warp_wait(smem_u32(&aux.full[stage]), phase, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t a0 = smem_u32(smem + stage * C::STAGE_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint32_t acc = (kb | kk) ? 1u : 0u;
+                        if constexpr (!SWAP) {
+                            tc_mma(d_tmem, sdesc_sw128(a0 + kk * 32), sdesc_sw128(a0 + C::A_BYTES + kk * 32), idesc,
+                                   acc);
+                        } else {
+                            const uint32_t b0 = a0 + C::NUM_A * C::A_BYTES;
+                            tc_mma(d_tmem, sdesc_sw128(a0 + kk * 32), sdesc_sw128(b0 + kk * 32), idesc, acc);
+                            if (SWIGLU)
+                                tc_mma(d_tmem + R, sdesc_sw128(a0 + C::A_BYTES + kk * 32), sdesc_sw128(b0 + kk * 32),
+                                       idesc, acc);
+                        }
+                    }
+                    tc_commit(smem_u32(&aux.empty[stage]));
+                }
+                __syncwarp();
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok) {
+                if (lane == 0) {
+                    *abort_flag = 1;
+                    set_status(p.status, DEV_TIMEOUT);
+                }
+                break;
+            }
+            if (lane == 0) tc_commit(smem_u32(&aux.tfull[buf]));
+            __syncwarp();
+        }
+        // all MMAs of this thread complete before tensor memory is freed
+        if (lane == 0) {
+            tc_commit(smem_u32(&aux.drain));
+            mbar_wait(smem_u32(&aux.drain), 0, abort_flag);
+        }
+        __syncwarp();
+    } else {
+        // ================= epilogue (warps 2..5 -> TMEM lane quarters 2,3,0,1)
+        const int q = warp & 3;
+        int j = 0;
+        for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x, ++j) {
+            const int buf = j & 1;
+            const uint32_t use = (uint32_t)(j >> 1);
+            if (!warp_wait(smem_u32(&aux.tfull[buf]), use & 1u, abort_flag)) {
+                if (lane == 0) {
+                    *abort_flag = 1;
+                    set_status(p.status, DEV_TIMEOUT);
+                }
+                break;
+            }
+            tc_fence_after();
+            int e, rb, cb;
+            decode_tile(aux, E, R, tile, e, rb, cb);
+            const int rows = min(R, aux.cnt[e] - rb * R);
+            const int64_t row0 = (int64_t)aux.off[e] + (int64_t)rb * R;
+            const uint32_t tb = tmem_base + (uint32_t)(buf * C::ACC) + ((uint32_t)(32 * q) << 16);
+            if constexpr (!SWAP) {
+                const int m = 32 * q + lane;  // activation row inside the tile
+                uint16_t* orow = p.out + (row0 + m) * p.ldo + (int64_t)cb * COLS;
+                const bool valid = m < rows;
+#pragma unroll 1
+                for (int c = 0; c < COLS; c += 32) {
+                    uint32_t g[32];
+                    tmem_ld32(tb + c, g);
+                    uint32_t pk[16];
+                    if constexpr (SWIGLU) {
+                        uint32_t u[32];
+                        tmem_ld32(tb + COLS + c, u);
+                        tmem_wait_ld(g);
+                        tmem_wait_ld(u);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            pk[i] = pack_bf16x2(silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
+                                                silu_mul(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1])));
+                    } else {
+                        tmem_wait_ld(g);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            pk[i] = pack_bf16x2(__uint_as_float(g[2 * i]), __uint_as_float(g[2 * i + 1]));
+                    }
+                    if (valid) {
+#pragma unroll
+                        for (int v = 0; v < 4; ++v)
+                            st16(orow + c + 8 * v, make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]));
+                    }
+                }
+            } else {
+                const int f = 32 * q + lane;  // weight row (output column) inside the tile
+                uint16_t* ocol = p.out + row0 * p.ldo + (int64_t)cb * 128 + f;
+#pragma unroll 1
+                for (int c = 0; c < rows; c += C::LDW) {
+                    uint32_t g[C::LDW];
+                    tmem_ld(tb + c, g);
+                    if constexpr (SWIGLU) {
+                        uint32_t u[C::LDW];
+                        tmem_ld(tb + R + c, u);
+                        tmem_wait_ld(g);
+                        tmem_wait_ld(u);
+#pragma unroll
+                        for (int i = 0; i < C::LDW; ++i)
+                            if (c + i < rows)
+                                ocol[(int64_t)(c + i) * p.ldo] = (uint16_t)f32_to_bf16_bits(
+                                    silu_mul(__uint_as_float(g[i]), __uint_as_float(u[i])));
+                    } else {
+                        tmem_wait_ld(g);
+#pragma unroll
+                        for (int i = 0; i < C::LDW; ++i)
+                            if (c + i < rows)
+                                ocol[(int64_t)(c + i) * p.ldo] = (uint16_t)f32_to_bf16_bits(__uint_as_float(g[i]));
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&aux.tempty[buf]));
+        }
+    }
+
+    // ---- teardown
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
+}
+
+// ----------------------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// bf16 matrix [rows][inner] (inner contiguous), box = 64 x box_rows, 128-byte swizzle
+static bool encode_2d(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {inner * 2};
+    cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <bool SWAP, bool SWIGLU, int R, int COLS>
+static cudaError_t run(const Ctx& c, const void* act, int S, const void* w1, const void* w2, const Args& a) {
+    using C = Cfg<SWAP, SWIGLU, R, COLS>;
+    auto kern = grouped_gemm_kernel<SWAP, SWIGLU, R, COLS>;
+    static bool attr_done[64] = {};
+    if (c.device < 0 || c.device >= 64) return cudaErrorInvalidDevice;
+    if (!attr_done[c.device]) {
+        cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        if (err != cudaSuccess) return err;
+        attr_done[c.device] = true;
+    }
+    CUtensorMap tm_act, tm_w1, tm_w2;
+    if (!encode_2d(&tm_act, act, (uint64_t)a.K, (uint64_t)S, (uint32_t)R)) return cudaErrorInvalidValue;
+    if (!encode_2d(&tm_w1, w1, (uint64_t)a.K, (uint64_t)a.E * a.n_out, (uint32_t)C::WBOX)) return cudaErrorInvalidValue;
+    if (!encode_2d(&tm_w2, SWIGLU ? w2 : w1, (uint64_t)a.K, (uint64_t)a.E * a.n_out, (uint32_t)C::WBOX))
+        return cudaErrorInvalidValue;
+    // upper bound on the tile count: sum_e ceil(cnt_e / R) <= S / R + E
+    const int64_t max_tiles = ((int64_t)S / R + a.E) * (a.n_out / COLS);
+    const int grid = (int)(max_tiles < c.num_sms ? max_tiles : c.num_sms);
+    if (grid <= 0) return cudaSuccess;
+    return launch(kern, dim3(grid), dim3(kThreads), (size_t)C::SMEM, c, tm_act, tm_w1, tm_w2, a);
+}
+
+// Rows-as-M when experts average at least 96 rows; otherwise weights-as-M with
+// the smallest row block that holds about twice the average.
+static int pick_rows(int S, int E) {
+    const int avg = E > 0 ? S / E : 0;
+    if (avg >= 96) return 0;
+    if (avg <= 8) return 16;
+    if (avg <= 16) return 32;
+    if (avg <= 32) return 64;
+    return 128;
+}
+
+}  // namespace tc
+
+cudaError_t launch_gate_up_bf16(const Ctx& c, const void* xp, const void* Wg, const void* Wu, const int32_t* counts,
+                                const int32_t* offsets, int S, int E, int d, int d_ff, void* h, int32_t* status) {
+    if (S == 0) return cudaSuccess;
+    tc::Args a{counts, offsets, E, d, d_ff, static_cast<uint16_t*>(h), (int64_t)d_ff, status};
+    switch (tc::pick_rows(S, E)) {
+        case 0: return tc::run<false, true, 128, 128>(c, xp, S, Wg, Wu, a);
+        case 16: return tc::run<true, true, 16, 128>(c, xp, S, Wg, Wu, a);
+        case 32: return tc::run<true, true, 32, 128>(c, xp, S, Wg, Wu, a);
+        case 64: return tc::run<true, true, 64, 128>(c, xp, S, Wg, Wu, a);
+        default: return tc::run<true, true, 128, 128>(c, xp, S, Wg, Wu, a);
+    }
+}
+
+cudaError_t launch_down_bf16(const Ctx& c, const void* h, const void* Wd, const int32_t* counts, const int32_t* offsets,
+                             int S, int E, int d, int d_ff, void* y, int32_t* status) {
+    if (S == 0) return cudaSuccess;
+    tc::Args a{counts, offsets, E, d_ff, d, static_cast<uint16_t*>(y), (int64_t)d, status};
+    switch (tc::pick_rows(S, E)) {
+        case 0:
+            if (d % 256 == 0) return tc::run<false, false, 128, 256>(c, h, S, Wd, nullptr, a);
+            return tc::run<false, false, 128, 128>(c, h, S, Wd, nullptr, a);
+        case 16: return tc::run<true, false, 16, 128>(c, h, S, Wd, nullptr, a);
+        case 32: return tc::run<true, false, 32, 128>(c, h, S, Wd, nullptr, a);
+        case 64: return tc::run<true, false, 64, 128>(c, h, S, Wd, nullptr, a);
+        default: return tc::run<true, false, 128, 128>(c, h, S, Wd, nullptr, a);
+    }
+}
+
+}  // namespace moe

@@ -1,0 +1,78 @@
+// Host-side launchers of the MoE layer kernels (internal to libmoe.so).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <utility>
+
+namespace moe {
+
+struct Ctx {
+    cudaStream_t stream;
+    int num_sms;
+    int device;
+};
+
+// Every kernel is launched with programmatic stream serialisation; each one
+// executes griddepcontrol.wait before it touches global memory, so it never
+// reads a predecessor's output early, and triggers its dependents as soon as
+// its own prologue is done.
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, const Ctx& c, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = c.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// ---- step 1: RMSNorm (norm_router.cu)
+cudaError_t launch_rmsnorm(const Ctx& c, const void* x, int x_dt, const float* gamma, int T, int d, float eps, void* v,
+                           int v_dt, float* rstd);
+
+// ---- step 2: router (norm_router.cu)
+struct RouterPlan {
+    int splitk;  // K split of the logits GEMM
+    int kchunk;  // K extent of one split (multiple of 32)
+    size_t partial_bytes;
+};
+RouterPlan plan_router(int T, int d, int E, int num_sms);
+// A operand: v (a_dt) when rstd == nullptr, else x (a_dt) * rstd[t] * gamma[j]
+cudaError_t launch_router_logits(const Ctx& c, const RouterPlan& p, const void* a, int a_dt, const float* rstd,
+                                 const float* gamma, const float* W_r, int T, int d, int E, float* partial);
+cudaError_t launch_router_topk(const Ctx& c, const RouterPlan& p, const float* partial, const float* b, int T, int E,
+                               int k, int32_t* idx, float* w, float* logits, float* margin);
+
+// ---- step 3: permutation (permute.cu)
+constexpr int kPermuteChunk = 256;
+inline size_t permute_ws_bytes(int T, int E) {
+    size_t nchunks = (size_t)(T + kPermuteChunk - 1) / kPermuteChunk;
+    return nchunks * (size_t)E * sizeof(int32_t);
+}
+cudaError_t launch_permute(const Ctx& c, const void* v, int v_dt, const int32_t* idx, int T, int d, int E, int k,
+                           int32_t* counts, int32_t* offsets, int32_t* slot_token, int32_t* token_slot, void* xp,
+                           int32_t* hist, int32_t* status);
+
+// ---- step 4: expert MLP (expert_tc.cu: bf16 tensor cores; expert_simt.cu: fp32)
+cudaError_t launch_gate_up_bf16(const Ctx& c, const void* xp, const void* Wg, const void* Wu, const int32_t* counts,
+                                const int32_t* offsets, int S, int E, int d, int d_ff, void* h, int32_t* status);
+cudaError_t launch_down_bf16(const Ctx& c, const void* h, const void* Wd, const int32_t* counts, const int32_t* offsets,
+                             int S, int E, int d, int d_ff, void* y, int32_t* status);
+cudaError_t launch_gate_up_f32(const Ctx& c, const float* xp, const float* Wg, const float* Wu, const int32_t* counts,
+                               const int32_t* offsets, int S, int E, int d, int d_ff, float* h);
+cudaError_t launch_down_f32(const Ctx& c, const float* h, const float* Wd, const int32_t* counts,
+                            const int32_t* offsets, int S, int E, int d, int d_ff, float* y);
+
+// ---- step 5: weighted un-permute + residual (combine.cu)
+cudaError_t launch_combine(const Ctx& c, const void* y, int y_dt, const int32_t* token_slot, const float* w,
+                           const void* res, int r_dt, int T, int d, int k, void* out, int out_dt);
+
+}  // namespace moe
