@@ -41,6 +41,9 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode", help="tiny | decode | prefill | skewed | block")
+    ap.add_argument("--shrink", type=int, default=1,
+                    help="divide T and E by this factor (same rows per expert, smaller device footprint); "
+                         "for ncu captures of the same kernels, never for reported numbers")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     a = ap.parse_args()
@@ -345,6 +348,8 @@ def main():
     import synth
 
     w = synth.WORKLOADS[a.workload]
+    if a.shrink > 1:
+        w = w.scaled(name=f"{w.name}/shrink{a.shrink}", T=max(1, w.T // a.shrink), E=max(w.top_k, w.E // a.shrink))
     if a.impl == "reference":
         return run_reference(a, w)
     return run_ours(a, w)
