@@ -1,6 +1,6 @@
 """Build ``libmoe.so`` in-tree with nvcc for sm_100a (B200).
 
-    python -m moe_layer_forward_b200.build [--force] [--ptxas-v]
+    python moe_layer_forward_b200/build.py [--force] [--ptxas-v]
 
 Each ``csrc/*.cu`` compiles to an object under ``_build/`` (skipped when up to
 date), then nvcc links the shared library next to this file.  The CUDA
