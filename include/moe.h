@@ -123,6 +123,32 @@ moe_status_t moe_permute(const void* v, moe_dtype_t v_dt, const int32_t* topk_id
                          void* xp, void* ws, size_t* ws_bytes, int32_t* dev_status, moe_stream_t stream);
 
 /*
+ * moe_permute without a workspace, for callers that cannot allocate device
+ * memory.  The pages have no counterpart: this is a convenience of this library.
+ *
+ * Some callers are handed only the tensors of the call and may not allocate on
+ * the device while it runs (e.g. an inference engine's plugin execute hook that
+ * owns a fixed memory pool, where an allocation would stall the stream or
+ * fragment the pool).  This call computes exactly what moe_permute computes,
+ * with the same kernels, but keeps their scratch (the per-chunk expert
+ * histogram) in a 256 KiB array inside the library that each GPU loading it
+ * holds until the process exits.  It calls no cudaMalloc/cudaFree.
+ *   - T must be <= MOE_PERMUTE_STATIC_MAX_TOKENS (65536), else
+ *     MOE_ERR_UNSUPPORTED; other arguments as for moe_permute.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls share the one array and nothing in it needs to start at zero
+ *     (every entry read is written earlier in the same call), but calls whose
+ *     work overlaps on the GPU (other streams, other host threads) race on it:
+ *     order them on one stream.
+ */
+#define MOE_PERMUTE_STATIC_MAX_TOKENS 65536
+moe_status_t moe_permute_static_ws(const void* v, moe_dtype_t v_dt, const int32_t* topk_idx, int32_t T, int32_t d,
+                                   int32_t E, int32_t k, int32_t* counts, int32_t* offsets, int32_t* slot_token,
+                                   int32_t* token_slot, void* xp, int32_t* dev_status, moe_stream_t stream);
+
+/*
  * Step 4, first half — gate/up projections with the SwiGLU product
  * [P1 §实际 MLP 计算策略: SiLU(X W_gate) ⊙ X W_up; §EP 路径: grouped GEMM]:
  *   h[r][f] = SiLU(sum_j xp[r][j] W_gate[e][f][j]) * (sum_j xp[r][j] W_up[e][f][j])

@@ -43,6 +43,7 @@ _sig = {
     "moe_rmsnorm": [_vp, _i32, _vp, _i32, _i32, _f32, _vp, _i32, _vp],
     "moe_router_topk": [_vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _szp, _vp],
     "moe_permute": [_vp, _i32, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _szp, _vp, _vp],
+    "moe_permute_static_ws": [_vp, _i32, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
     "moe_expert_gate_up": [_vp, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp],
     "moe_expert_down": [_vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp],
     "moe_grouped_swiglu": [_vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp],
@@ -134,6 +135,20 @@ def moe_permute(v, topk_idx, E: int, counts, offsets, slot_token, token_slot, xp
         ws = _ws(lambda w, n: _check("moe_permute", call(w, n)), v.device)
     n = ctypes.c_size_t(ws.numel())
     _check("moe_permute", call(_p(ws), ctypes.byref(n)))
+
+
+def moe_permute_static_ws(v, topk_idx, E: int, counts, offsets, slot_token, token_slot, xp,
+                          dev_status=None) -> None:
+    """moe_permute for callers that cannot allocate: the library keeps the scratch itself.
+
+    Same results as ``moe_permute``; needs no workspace (T <= 65536).  Calls that
+    overlap on the GPU share that scratch and race, so keep them on one stream.
+    """
+    T, d = v.shape
+    k = topk_idx.shape[1]
+    _check("moe_permute_static_ws", _lib.moe_permute_static_ws(_p(v), _dt(v), _p(topk_idx), T, d, E, k, _p(counts),
+                                                               _p(offsets), _p(slot_token), _p(token_slot), _p(xp),
+                                                               _p(dev_status), _stream(v.device)))
 
 
 def moe_expert_gate_up(xp, W_gate, W_up, counts, offsets, h, dev_status=None) -> None:
