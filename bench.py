@@ -29,7 +29,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer tokens/s at 1 B200; % of HBM (decode) / BF16 tensor (prefill) roofline"
 L2_BYTES = 126 * 1024 * 1024
-LAUNCHES_PER_STEP = 10  # rmsnorm, router logits, router top-k, 4 permute kernels, gate/up, down, combine
+LAUNCHES_PER_STEP = 11  # rmsnorm, W_r split, router logits, router top-k, 4 permute kernels, gate/up, down, combine
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "roofline_traffic.json")
 GEMM_SRC = os.path.join(ROOT, "moe_layer_forward_b200", "csrc", "expert_tc.cu")
 

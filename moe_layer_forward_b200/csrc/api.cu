@@ -144,13 +144,15 @@ moe_status_t moe_router_topk(const void* v, moe_dtype_t v_dt, const float* W_r, 
     const RouterPlan plan = plan_router(T, d, E, c.num_sms);
     Carve cv(nullptr);
     cv.take(plan.partial_bytes);
+    cv.take(plan.wsplit_bytes);
     bool query = false;
     st = check_ws(ws, ws_bytes, cv.off, &query);
     if (st != MOE_OK || query || T == 0) return st;
     if (!v || !W_r || !b || !topk_idx || !topk_w || !aligned16(v) || !aligned16(W_r)) return MOE_ERR_INVALID_ARG;
     Carve w(ws);
     float* partial = static_cast<float*>(w.take(plan.partial_bytes));
-    st = cuda_status(launch_router_logits(c, plan, v, v_dt, nullptr, nullptr, W_r, T, d, E, partial));
+    float* wsplit = static_cast<float*>(w.take(plan.wsplit_bytes));
+    st = cuda_status(launch_router_logits(c, plan, v, v_dt, nullptr, nullptr, W_r, T, d, E, partial, wsplit, nullptr));
     if (st != MOE_OK) return st;
     return cuda_status(launch_router_topk(c, plan, partial, b, T, E, k, topk_idx, topk_w, logits, margin));
 }
@@ -263,6 +265,7 @@ moe_status_t moe_forward(const moe_shape_t* shape, const moe_weights_t* wts, con
     void* v = cv.take((size_t)T * d * es);
     float* rstd = static_cast<float*>(cv.take((size_t)T * sizeof(float)));
     float* partial = static_cast<float*>(cv.take(plan.partial_bytes));
+    float* wsplit = static_cast<float*>(cv.take(plan.wsplit_bytes));
     // routing is kept in the workspace unless the caller asks for it (the size never depends on that)
     int32_t* idx_ws = static_cast<int32_t*>(cv.take((size_t)S * sizeof(int32_t)));
     float* wgt_ws = static_cast<float*>(cv.take((size_t)S * sizeof(float)));
@@ -297,7 +300,8 @@ moe_status_t moe_forward(const moe_shape_t* shape, const moe_weights_t* wts, con
     st = cuda_status(launch_rmsnorm(c, x, xdt, wts->gamma, T, d, shape->eps, v, wdt, rstd));
     if (st != MOE_OK) return st;
     // 2. router on the unrounded fp32 normalised rows (x * rstd * gamma formed in the GEMM)
-    st = cuda_status(launch_router_logits(c, plan, x, xdt, rstd, wts->gamma, wts->W_r, T, d, E, partial));
+    st = cuda_status(
+        launch_router_logits(c, plan, x, xdt, rstd, wts->gamma, wts->W_r, T, d, E, partial, wsplit, dev_status));
     if (st != MOE_OK) return st;
     st = cuda_status(launch_router_topk(c, plan, partial, wts->b, T, E, k, idx, wgt, logits, nullptr));
     if (st != MOE_OK) return st;

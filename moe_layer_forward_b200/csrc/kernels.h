@@ -38,16 +38,18 @@ cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
 cudaError_t launch_rmsnorm(const Ctx& c, const void* x, int x_dt, const float* gamma, int T, int d, float eps, void* v,
                            int v_dt, float* rstd);
 
-// ---- step 2: router (norm_router.cu)
+// ---- step 2: router (router_tc.cu: logits on tensor cores; norm_router.cu: top-k)
 struct RouterPlan {
-    int splitk;  // K split of the logits GEMM
-    int kchunk;  // K extent of one split (multiple of 32)
-    size_t partial_bytes;
+    int splitk;           // K split of the logits GEMM
+    int kchunk;           // K extent of one split (multiple of 32)
+    size_t partial_bytes; // [splitk][T][E] fp32 partial logits
+    size_t wsplit_bytes;  // W_r split into tf32 hi / lo terms
 };
 RouterPlan plan_router(int T, int d, int E, int num_sms);
 // A operand: v (a_dt) when rstd == nullptr, else x (a_dt) * rstd[t] * gamma[j]
 cudaError_t launch_router_logits(const Ctx& c, const RouterPlan& p, const void* a, int a_dt, const float* rstd,
-                                 const float* gamma, const float* W_r, int T, int d, int E, float* partial);
+                                 const float* gamma, const float* W_r, int T, int d, int E, float* partial,
+                                 float* wsplit, int32_t* status);
 cudaError_t launch_router_topk(const Ctx& c, const RouterPlan& p, const float* partial, const float* b, int T, int E,
                                int k, int32_t* idx, float* w, float* logits, float* margin);
 
