@@ -450,6 +450,7 @@ static int pick_rows(int S, int E) {
 cudaError_t launch_gate_up_bf16(const Ctx& c, const void* xp, const void* Wg, const void* Wu, const int32_t* counts,
                                 const int32_t* offsets, int S, int E, int d, int d_ff, void* h, int32_t* status) {
     if (S == 0) return cudaSuccess;
+    if (use_pair_gemm(S, E, 256)) return launch_gate_up_bf16_pair(c, xp, Wg, Wu, counts, offsets, S, E, d, d_ff, h, status);
     tc::Args a{counts, offsets, E, d, d_ff, static_cast<uint16_t*>(h), (int64_t)d_ff, status};
     switch (tc::pick_rows(S, E)) {
         case 0: return tc::run<false, true, 128, 128>(c, xp, S, Wg, Wu, a);
@@ -463,6 +464,7 @@ cudaError_t launch_gate_up_bf16(const Ctx& c, const void* xp, const void* Wg, co
 cudaError_t launch_down_bf16(const Ctx& c, const void* h, const void* Wd, const int32_t* counts, const int32_t* offsets,
                              int S, int E, int d, int d_ff, void* y, int32_t* status) {
     if (S == 0) return cudaSuccess;
+    if (use_pair_gemm(S, E, d)) return launch_down_bf16_pair(c, h, Wd, counts, offsets, S, E, d, d_ff, y, status);
     tc::Args a{counts, offsets, E, d_ff, d, static_cast<uint16_t*>(y), (int64_t)d, status};
     switch (tc::pick_rows(S, E)) {
         case 0:

@@ -68,6 +68,13 @@ cudaError_t launch_gate_up_bf16(const Ctx& c, const void* xp, const void* Wg, co
                                 const int32_t* offsets, int S, int E, int d, int d_ff, void* h, int32_t* status);
 cudaError_t launch_down_bf16(const Ctx& c, const void* h, const void* Wd, const int32_t* counts, const int32_t* offsets,
                              int S, int E, int d, int d_ff, void* y, int32_t* status);
+// CTA-pair (cta_group::2) variants for experts with many rows each (expert_tc2.cu)
+bool use_pair_gemm(int S, int E, int n_out);
+cudaError_t launch_gate_up_bf16_pair(const Ctx& c, const void* xp, const void* Wg, const void* Wu,
+                                     const int32_t* counts, const int32_t* offsets, int S, int E, int d, int d_ff,
+                                     void* h, int32_t* status);
+cudaError_t launch_down_bf16_pair(const Ctx& c, const void* h, const void* Wd, const int32_t* counts,
+                                  const int32_t* offsets, int S, int E, int d, int d_ff, void* y, int32_t* status);
 cudaError_t launch_gate_up_f32(const Ctx& c, const float* xp, const float* Wg, const float* Wu, const int32_t* counts,
                                const int32_t* offsets, int S, int E, int d, int d_ff, float* h);
 cudaError_t launch_down_f32(const Ctx& c, const float* h, const float* Wd, const int32_t* counts,

@@ -166,13 +166,16 @@ def _segments(counts):
 
 
 # row counts per expert chosen to reach each tile arrangement (average rows per expert decides it):
-#   weights-as-M with 16/32/64/128-row blocks, and rows-as-M; each has empty experts and ragged tails
+#   weights-as-M with 16/32/64/128-row blocks, rows-as-M on one CTA, and rows-as-M on CTA pairs
+#   (256-row blocks, including a block whose second CTA has one row or none); each has empty experts
+#   and ragged tails
 COUNT_CASES = {
     "w16": [0, 1, 3, 8, 16, 17, 33, 5, 0, 9, 2, 7, 4, 6, 10, 7],        # avg 8
     "w32": [12, 0, 16, 31, 33, 9, 20, 15, 4, 14, 18, 2, 16, 11, 13, 10],  # avg 14
     "w64": [0, 64, 65, 20, 1, 40, 30, 37],                             # avg 32
     "w128": [129, 0, 60, 45, 33, 90, 7, 100],                          # avg 58
     "rows": [0, 1, 127, 128, 129, 300, 0, 290],                        # avg 122
+    "pairs": [0, 255, 256, 257, 2900, 1024, 1, 1513],                  # avg 775: CTA-pair kernel, 256-row blocks
 }
 
 
@@ -220,7 +223,7 @@ def test_expert_down_bf16(moe, case, d, d_ff):
     assert_close_rounded(y, ref)
 
 
-@pytest.mark.parametrize("case", ["w16", "w64", "rows"])
+@pytest.mark.parametrize("case", ["w16", "w64", "rows", "pairs"])
 def test_expert_down_integer_inputs_bit_exact(moe, case):
     # entries in {-1, 0, 1}: every fp32 partial sum is an integer below 2^24 and |y| <= d_ff = 256, so the
     # tensor-core result rounds to bf16 exactly and must equal the oracle bit for bit
@@ -251,7 +254,7 @@ def test_expert_mlp_f32(moe, case):
     assert_close_rounded(y, y_ref, rel=1e-4, rms_frac=1e-5)
 
 
-@pytest.mark.parametrize("case", ["w16", "w32", "rows"])
+@pytest.mark.parametrize("case", ["w16", "w32", "rows", "pairs"])
 def test_grouped_swiglu_bf16_matches_oracle(moe, case):
     d, d_ff = 256, 256
     counts, offsets, xp, Wg, Wu, Wd = _expert_inputs(case, d, d_ff, seed=304)
