@@ -31,7 +31,7 @@ METRIC = "MoE-layer tokens/s at 1 B200; % of HBM (decode) / BF16 tensor (prefill
 L2_BYTES = 126 * 1024 * 1024
 LAUNCHES_PER_STEP = 11  # rmsnorm, W_r split, router logits, router top-k, 4 permute kernels, gate/up, down, combine
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "roofline_traffic.json")
-GEMM_SRC = os.path.join(ROOT, "moe_layer_forward_b200", "csrc", "expert_tc.cu")
+GEMM_SRC = [os.path.join(ROOT, "moe_layer_forward_b200", "csrc", f) for f in ("expert_tc.cu", "tc_ptx.cuh")]
 
 
 def parse():
@@ -54,6 +54,26 @@ def parse():
 def dist_env():
     return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(
         os.environ.get("LOCAL_RANK", "0"))
+
+
+def reduce_max_fn(dist, device):
+    """max over ranks of a float (identity on one rank); the only cross-rank operation of a replica run"""
+    import torch
+
+    def reduce_max(v: float) -> float:
+        if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    return reduce_max
+
+
+def aggregate(local_ms: float, units_per_rank: int, steps: int, world: int, reduce_max):
+    """(whole-job units/s, ms per step): every rank processed units_per_rank per step; time = slowest rank"""
+    ms = reduce_max(local_ms)
+    return world * units_per_rank * steps / (ms / 1000.0), ms / steps
 
 
 def peaks():
@@ -116,7 +136,7 @@ def traffic_for(workload: str):
     if not os.path.exists(TRAFFIC_FILE):
         return None
     j = json.load(open(TRAFFIC_FILE))
-    sha = hashlib.sha256(open(GEMM_SRC, "rb").read()).hexdigest()[:16]
+    sha = hashlib.sha256(b"".join(open(f, "rb").read() for f in GEMM_SRC)).hexdigest()[:16]
     e = j.get(workload)
     if not e or e.get("source_sha") != sha:
         return None
@@ -141,8 +161,8 @@ def cpu_baseline(I, w):
     n = int(max(1, min(256, 15.0 / max(t1, 1e-3))))
     v, dt = oracle_tokens_per_s(I, w, n, start=1)
     return {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n} of {w.T} tokens of the {w.name} workload, whole layer per token in fp64 "
-                      f"(single-threaded C, {dt:.1f} s)"}
+            "sample": f"{n} token rows cycling through the {w.T} of the {w.name} workload, whole layer per "
+                      f"token in fp64 (single-threaded C, {dt:.1f} s)"}
 
 
 def run_reference(a, w):
@@ -214,12 +234,7 @@ def run_ours(a, w):
             dist.barrier()
         torch.cuda.synchronize()
 
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    max_over_ranks = reduce_max_fn(dist, dev)
 
     for _ in range(a.warmup):
         step()
@@ -236,9 +251,7 @@ def run_ours(a, w):
             step()
         e1.record()
         barrier()
-    ms = max_over_ranks(e0.elapsed_time(e1))
-    ms_per_step = ms / a.steps
-    value = world * T * a.steps / (ms / 1000.0)
+    value, ms_per_step = aggregate(e0.elapsed_time(e1), T, a.steps, world, max_over_ranks)
     if status.item() != 0:
         raise RuntimeError(f"device status {status.item()} in the timed region")
 
@@ -320,8 +333,8 @@ def run_ours(a, w):
             torch.cuda.current_stream().synchronize()  # the host reads this step's result
         f1.record()
         barrier()
-        ems = max_over_ranks(f0.elapsed_time(f1))
-        e2e = {"value": world * T * a.steps / (ems / 1000.0), "unit": "tokens/s",
+        e2e_value, _ = aggregate(f0.elapsed_time(f1), T, a.steps, world, max_over_ranks)
+        e2e = {"value": e2e_value, "unit": "tokens/s",
                "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
                "d2h_bytes_per_step": out_host.numel() * out_host.element_size()}
 

@@ -1,0 +1,92 @@
+"""The N > 1 path of the benchmark, on CPU with two gloo ranks.
+
+The layer shards by tokens: every rank runs an independent replica on its own
+tokens, so the only cross-rank operations are a barrier and the max over ranks
+of the timed duration.  These tests run that logic in two spawned processes.
+"""
+import os
+import socket
+import sys
+import tempfile
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank: int, world: int, port: int, outdir: str):
+    sys.path.insert(0, ROOT)
+    import datetime
+
+    import torch.distributed as dist
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    import bench
+    import oracle
+    import synth
+
+    # timing: rank r took 10 * (r + 1) ms for 5 steps of 128 tokens; the job time is the slowest rank's
+    value, ms_per_step = bench.aggregate(10.0 * (rank + 1), 128, 5, world, bench.reduce_max_fn(dist, "cpu"))
+    dist.barrier()
+    # replicas: each rank computes the layer on its own shard of the tokens
+    w = synth.Workload("shard", 12, 64, 16, 32, x_dtype=torch.float32, w_dtype=torch.float32,
+                       out_dtype=torch.float32, seed=31)
+    I = synth.make_layer_inputs(w)
+    shard = I["x"][rank::world]
+    out = oracle.moe_layer(shard, I["gamma"], I["W_r"], I["b"], I["W_gate"], I["W_up"], I["W_down"])["out"]
+    torch.save({"value": value, "ms_per_step": ms_per_step, "out": out}, os.path.join(outdir, f"r{rank}.pt"))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_aggregate_with_the_slowest_rank_and_shard_tokens():
+    world = 2
+    with tempfile.TemporaryDirectory() as d:
+        mp.start_processes(_worker, args=(world, _free_port(), d), nprocs=world, join=True, start_method="spawn")
+        r = [torch.load(os.path.join(d, f"r{k}.pt")) for k in range(world)]
+    for k in range(world):
+        assert r[k]["value"] == pytest.approx(world * 128 * 5 / 0.020)  # slowest rank: 20 ms
+        assert r[k]["ms_per_step"] == pytest.approx(4.0)
+    # concatenating the ranks' shards reproduces the single-process layer (no data-path collective needed)
+    sys.path.insert(0, ROOT)
+    import oracle
+    import synth
+
+    w = synth.Workload("shard", 12, 64, 16, 32, x_dtype=torch.float32, w_dtype=torch.float32,
+                       out_dtype=torch.float32, seed=31)
+    I = synth.make_layer_inputs(w)
+    full = oracle.moe_layer(I["x"], I["gamma"], I["W_r"], I["b"], I["W_gate"], I["W_up"], I["W_down"])["out"]
+    merged = torch.empty_like(full)
+    for k in range(world):
+        merged[k::world] = r[k]["out"]
+    assert torch.equal(merged, full)
+
+
+def test_single_rank_aggregate_is_local():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    value, ms = bench.aggregate(8.0, 100, 4, 1, lambda v: v)
+    assert value == pytest.approx(100 * 4 / 0.008) and ms == pytest.approx(2.0)
+
+
+def test_reference_arm_runs_only_on_rank_zero(monkeypatch):
+    sys.path.insert(0, ROOT)
+    import argparse
+
+    import bench
+    import synth
+
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    a = argparse.Namespace(steps=2, warmup=3, gpus=2)
+    assert bench.run_reference(a, synth.WORKLOADS["decode"]) == 0  # returns at once, no inputs generated
