@@ -211,6 +211,13 @@ moe_status_t moe_forward(const moe_shape_t* shape, const moe_weights_t* weights,
 /* Static text for a status code. */
 const char* moe_status_string(moe_status_t status);
 
+/* Number of kernels the library has enqueued in this process since it was
+ * loaded, over all entry points, streams and threads (successful launches
+ * only; a launch that returned an error is not counted).  Not part of any
+ * method on the pages: it lets a caller check how many device launches a call
+ * made, e.g. to count the kernels of a timed loop.  Never fails. */
+uint64_t moe_kernel_launches(void);
+
 /* ABI version of this header (bumped on any incompatible change). */
 #define MOE_ABI_VERSION 1
 int32_t moe_abi_version(void);

@@ -58,6 +58,7 @@ for _name, _args in _sig.items():
 _lib.moe_status_string.argtypes = [ctypes.c_int]
 _lib.moe_status_string.restype = ctypes.c_char_p
 _lib.moe_abi_version.restype = ctypes.c_int32
+_lib.moe_kernel_launches.restype = ctypes.c_uint64
 
 
 class MoEError(RuntimeError):
@@ -101,6 +102,11 @@ def _ws(query, device) -> torch.Tensor:
 
 def abi_version() -> int:
     return int(_lib.moe_abi_version())
+
+
+def kernel_launches() -> int:
+    """Kernels the library has enqueued in this process so far (all entry points)."""
+    return int(_lib.moe_kernel_launches())
 
 
 def moe_rmsnorm(x: torch.Tensor, gamma: torch.Tensor, eps: float, v: torch.Tensor) -> None:

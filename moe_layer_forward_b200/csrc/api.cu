@@ -7,6 +7,10 @@
 #include "kernels.h"
 #include "moe.h"
 
+namespace moe {
+std::atomic<uint64_t> g_kernel_launches{0};
+}  // namespace moe
+
 using namespace moe;
 
 namespace {
@@ -119,6 +123,8 @@ const char* moe_status_string(moe_status_t s) {
 }
 
 int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+uint64_t moe_kernel_launches(void) { return moe::g_kernel_launches.load(std::memory_order_relaxed); }
 
 moe_status_t moe_rmsnorm(const void* x, moe_dtype_t x_dt, const float* gamma, int32_t T, int32_t d, float eps,
                          void* v, moe_dtype_t v_dt, moe_stream_t stream) {

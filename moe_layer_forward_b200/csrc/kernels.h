@@ -5,9 +5,13 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <utility>
 
 namespace moe {
+
+// Kernels this library has enqueued in this process (successful launches only).
+extern std::atomic<uint64_t> g_kernel_launches;
 
 struct Ctx {
     cudaStream_t stream;
@@ -31,7 +35,9 @@ cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+    const cudaError_t err = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+    if (err == cudaSuccess) g_kernel_launches.fetch_add(1, std::memory_order_relaxed);
+    return err;
 }
 
 // ---- step 1: RMSNorm (norm_router.cu)

@@ -55,6 +55,14 @@ def test_status_strings_and_version(lib):
     assert lib.moe_abi_version() == 1
 
 
+def test_launch_counter_counts_no_rejected_call(lib):
+    # arguments rejected on the host enqueue nothing, so the counter stays where it was
+    lib.moe_kernel_launches.restype = ctypes.c_uint64
+    n0 = lib.moe_kernel_launches()
+    assert lib.moe_rmsnorm(None, 1, None, -1, 64, ctypes.c_float(1e-5), None, 1, None) != 0
+    assert lib.moe_kernel_launches() == n0
+
+
 def test_library_does_not_link_the_oracle():
     out = subprocess.run(["nm", "-D", LIB], capture_output=True, text=True, check=True).stdout
     assert "oracle_" not in out

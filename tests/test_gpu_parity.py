@@ -169,13 +169,18 @@ def _segments(counts):
 #   weights-as-M with 16/32/64/128-row blocks, rows-as-M on one CTA, and rows-as-M on CTA pairs
 #   (256-row blocks, including a block whose second CTA has one row or none); each has empty experts
 #   and ragged tails
+# Per-expert row counts.  The name says which GEMM arrangement the average selects: token rows
+# staged per tile (16/32/64/128, about 3x the average) on one CTA, or CTA pairs with 256-row
+# blocks ("pairs", from 768 rows per expert).
 COUNT_CASES = {
-    "w16": [0, 1, 3, 8, 16, 17, 33, 5, 0, 9, 2, 7, 4, 6, 10, 7],        # avg 8
-    "w32": [12, 0, 16, 31, 33, 9, 20, 15, 4, 14, 18, 2, 16, 11, 13, 10],  # avg 14
-    "w64": [0, 64, 65, 20, 1, 40, 30, 37],                             # avg 32
-    "w128": [129, 0, 60, 45, 33, 90, 7, 100],                          # avg 58
-    "rows": [0, 1, 127, 128, 129, 300, 0, 290],                        # avg 122
-    "pairs": [0, 255, 256, 257, 2900, 1024, 1, 1513],                  # avg 775: CTA-pair kernel, 256-row blocks
+    "ra16": [0, 1, 3, 8, 16, 17, 5, 0, 2, 2, 7, 4, 1, 1, 2, 3],            # avg 4.5
+    "ra32": [0, 1, 3, 8, 16, 17, 33, 5, 0, 9, 2, 7, 4, 6, 10, 7],         # avg 8
+    "ra64": [12, 0, 16, 31, 33, 9, 20, 15, 4, 14, 18, 2, 16, 11, 13, 10],  # avg 14
+    "ra128": [0, 64, 65, 20, 1, 40, 30, 37],                              # avg 32
+    "ra128b": [129, 0, 60, 45, 33, 90, 7, 100],                           # avg 58
+    "rows": [0, 1, 127, 128, 129, 300, 0, 290],                           # avg 122
+    "rows256": [0, 1, 128, 129, 256, 257, 384, 511, 512, 640, 0, 300],    # avg 260: remainders 0/1/128/129/255
+    "pairs": [0, 255, 256, 257, 2900, 1024, 1, 1513],                     # avg 775
 }
 
 
@@ -223,7 +228,7 @@ def test_expert_down_bf16(moe, case, d, d_ff):
     assert_close_rounded(y, ref)
 
 
-@pytest.mark.parametrize("case", ["w16", "w64", "rows", "pairs"])
+@pytest.mark.parametrize("case", ["ra16", "ra128", "rows", "rows256", "pairs"])
 def test_expert_down_integer_inputs_bit_exact(moe, case):
     # entries in {-1, 0, 1}: every fp32 partial sum is an integer below 2^24 and |y| <= d_ff = 256, so the
     # tensor-core result rounds to bf16 exactly and must equal the oracle bit for bit
@@ -241,7 +246,7 @@ def test_expert_down_integer_inputs_bit_exact(moe, case):
     assert torch.equal(y.cpu().double(), ref)
 
 
-@pytest.mark.parametrize("case", ["w16", "rows"])
+@pytest.mark.parametrize("case", ["ra32", "rows"])
 def test_expert_mlp_f32(moe, case):
     d, d_ff = 64, 96
     counts, offsets, xp, Wg, Wu, Wd = _expert_inputs(case, d, d_ff, torch.float32, 303)
@@ -254,7 +259,7 @@ def test_expert_mlp_f32(moe, case):
     assert_close_rounded(y, y_ref, rel=1e-4, rms_frac=1e-5)
 
 
-@pytest.mark.parametrize("case", ["w16", "w32", "rows", "pairs"])
+@pytest.mark.parametrize("case", ["ra32", "ra64", "rows", "rows256", "pairs"])
 def test_grouped_swiglu_bf16_matches_oracle(moe, case):
     d, d_ff = 256, 256
     counts, offsets, xp, Wg, Wu, Wd = _expert_inputs(case, d, d_ff, seed=304)
@@ -398,6 +403,20 @@ def test_forward_workspace_too_small_is_rejected(moe):
     with pytest.raises(moe.MoEError) as ei:
         moe.moe_forward(I["x"], I["gamma"], I["W_r"], I["b"], I["W_gate"], I["W_up"], I["W_down"], out, ws=ws)
     assert ei.value.status == 3
+
+
+def test_forward_launch_count_is_reported_and_stable(moe):
+    # the library's own launch counter: one forward enqueues the same nonzero number of kernels each time
+    w = synth.Workload("count", 32, 256, 16, 128)
+    I = {n: cuda(t) for n, t in synth.make_layer_inputs(w).items()}
+    out = torch.empty((32, 256), dtype=torch.bfloat16, device=DEV)
+    n = []
+    for _ in range(3):
+        n0 = moe.kernel_launches()
+        moe.moe_forward(I["x"], I["gamma"], I["W_r"], I["b"], I["W_gate"], I["W_up"], I["W_down"], out)
+        n.append(moe.kernel_launches() - n0)
+    torch.cuda.synchronize()
+    assert n[0] > 0 and n[0] == n[1] == n[2]
 
 
 # --------------------------------------------------------------------------- full-size workloads (sampled)
