@@ -10,19 +10,28 @@
 // One persistent kernel template covers both halves of the expert MLP:
 //   gate/up: h = SiLU(xp W_gate^T) ⊙ (xp W_up^T)   (SwiGLU fused in the epilogue)
 //   down:    y = h W_down^T
-// A work tile is (expert e, row block rb of RA rows, column block cb).  The
-// MMA is always M = 128 rows x N = 256 weight rows (gate 128 | up 128
-// stacked, or 256 down rows) x K = 16: on B200 an M = 128 MMA takes the same
-// time for every N from 16 to 256 (86 ns per SM), so weights go on N, where a
-// few tokens per expert still consume 8 KB of weights per instruction.  When
-// experts have few rows (decode), only RA = 16/32/64 token rows are loaded
-// per stage; the MMA's remaining A rows read whatever follows in shared
-// memory, which only affects accumulator rows that are never stored.
-// Tiles are numbered expert-major, then column block, then row block, and
-// CTAs take tiles tile = blockIdx.x + i * gridDim.x, so the row blocks that
-// share a weight tile run side by side and read it from L2 once.  The
-// per-expert row counts live only on the device; every CTA turns them into a
-// tile prefix sum in shared memory (no host sync).
+// A work tile is (expert e, row block rb of R rows, column block cb).  Tiles
+// are numbered expert-major, then column block, then row block, and CTAs take
+// tiles tile = blockIdx.x + i * gridDim.x, so the row blocks that share a
+// weight tile run side by side and read it from L2 once.  The per-expert row
+// counts live only on the device; every CTA turns them into a tile prefix
+// sum in shared memory (no host sync).
+//
+// On B200 an M = 128 MMA takes the same time (~86 ns per K = 16 on one SM)
+// for every N from 16 to 256, and an M = 64 one as long as M = 128, so a
+// tile's cost is set by its instruction count, not its useful rows.  Two
+// operand arrangements:
+//   rows-as-M: MMA M = 128 token rows x N = 256 weight rows (gate 128 | up
+//     128 stacked, or 256 down rows).  Only R = 16/32/64/128 token rows are
+//     staged per K slice; the rest of the M = 128 operand reads whatever
+//     follows in shared memory and lands in accumulator rows that are never
+//     stored.  With few rows per expert one MMA still consumes 8 KB of
+//     weights, so the kernel streams weights at HBM speed.
+//   weights-as-M (gate/up with few rows per expert): M = 128 gate rows and
+//     128 up rows in two MMAs, N = the expert's rows rounded up to 16 (<= R).
+//     Measured at 8 rows per expert it runs gate/up ~4% faster than
+//     rows-as-M; for down, whose weight tile is one 128-row operand, it
+//     leaves the tensor pipe co-limiting and rows-as-M is ~30% faster.
 //
 // Warp roles (192 threads, 1 CTA per SM):
 //   warp 0      TMA producer: a STAGES-deep ring of 64-wide K slices (128-byte
@@ -31,9 +40,8 @@
 //               (4 x K=16 per stage) and tcgen05.commit to release each stage
 //               and to publish a finished accumulator.
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator (each warp its 32 TMEM
-//               lanes = 32 tile rows), SiLU(g)*u in fp32, bf16 16-byte stores.
-//               Two accumulator buffers let the epilogue of one tile overlap
-//               the next tile's MMAs.
+//               lanes), SiLU(g)*u in fp32, bf16 stores.  Two accumulator
+//               buffers let the epilogue of one tile overlap the next tile's MMAs.
 // Every wait is bounded (globaltimer); a wait that gives up raises
 // DEV_TIMEOUT in the status word and all roles unwind, drain in-flight copies
 // and MMAs, free tensor memory and exit.
@@ -54,24 +62,32 @@ constexpr int kSmemLimit = 232448;              // 227 KB opt-in per CTA
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
 
 // ----------------------------------------------------------------------------- configuration
-template <bool SWIGLU, int RA, int COLS>
+template <bool SWAP, bool SWIGLU, int R, int COLS>
 struct Cfg {
-    static_assert(RA == 16 || RA == 32 || RA == 64 || RA == 128, "rows per tile");
-    static_assert(!SWIGLU || COLS == 128, "gate/up tiles cover 128 features (N = 256)");
-    static constexpr int MMA_N = SWIGLU ? 2 * COLS : COLS;
-    static_assert(MMA_N == 128 || MMA_N == 256, "MMA N");
-    static constexpr int A_BYTES = RA * 128;      // token rows staged per K slice
-    static constexpr int B_BYTES = MMA_N * 128;   // weight rows staged per K slice
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static_assert(STAGE_BYTES >= 128 * 128, "the M = 128 operand read stays inside its stage");
-    static constexpr int WBOX = SWIGLU ? 128 : COLS;  // weight rows per TMA box
-    static constexpr int ACC = MMA_N;                 // accumulator columns per buffer
-    static constexpr int TMEM_COLS = (2 * ACC <= 256) ? 256 : 512;
+    // SWAP = weights are the MMA's A operand (M = 128 weight rows), activations B (N <= R).
+    static_assert(!SWAP || COLS == 128, "weights-as-M tiles cover 128 weight rows");
+    static_assert(R == 16 || R == 32 || R == 64 || R == 128, "row block");
+    static constexpr int MMA_N = SWAP ? R : (SWIGLU ? 2 * COLS : COLS);
+    static_assert(MMA_N % 16 == 0 && MMA_N <= 256, "MMA N for M = 128");
+    static constexpr int A_ROWS = SWAP ? 128 : R;
+    static constexpr int NUM_A = (SWAP && SWIGLU) ? 2 : 1;
+    static constexpr int B_ROWS = SWAP ? R : MMA_N;
+    static constexpr int A_BYTES = A_ROWS * 128;
+    static constexpr int B_BYTES = B_ROWS * 128;
+    static constexpr int STAGE_BYTES = NUM_A * A_BYTES + B_BYTES;
+    // rows-as-M reads 128 A rows from the stage start: they must stay inside the stage
+    static_assert(SWAP || STAGE_BYTES >= 128 * 128, "M = 128 operand inside its stage");
+    static constexpr int WBOX = SWAP ? 128 : (SWIGLU ? 128 : COLS);  // weight rows per TMA box
+    // accumulator columns per buffer: SWAP+SWIGLU keeps gate and up side by side
+    static constexpr int ACC = SWAP ? (SWIGLU ? 2 * R : R) : MMA_N;
+    static constexpr int TMEM_COLS = (2 * ACC <= 32) ? 32 : (2 * ACC <= 64) ? 64 : (2 * ACC <= 128) ? 128 : (2 * ACC <= 256) ? 256 : 512;
+    static_assert(2 * ACC <= 512, "two accumulator buffers must fit in 512 TMEM columns");
     static constexpr int AUX_BYTES = 4096;  // barriers, tile tables
     static constexpr int STAGES_MAX = (kSmemLimit - 1024 - AUX_BYTES) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_MAX > 12 ? 12 : STAGES_MAX;
     static_assert(STAGES >= 2, "pipeline depth");
     static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + AUX_BYTES;
+    static constexpr int LDW = R < 32 ? R : 32;  // TMEM columns per tcgen05.ld in the weights-as-M epilogue
 };
 
 struct Args {
@@ -111,12 +127,11 @@ __device__ __forceinline__ void decode_tile(const Aux& a, int E, int R, int tile
     rb = local - cb * nrb;
 }
 
-template <bool SWIGLU, int RA, int COLS>
+template <bool SWAP, bool SWIGLU, int R, int COLS>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_w1,
                         const __grid_constant__ CUtensorMap tm_w2, const Args p) {
-    using C = Cfg<SWIGLU, RA, COLS>;
-    constexpr int R = RA;
+    using C = Cfg<SWAP, SWIGLU, R, COLS>;
     constexpr int STAGES = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -206,9 +221,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint8_t* st = smem + stage * C::STAGE_BYTES;
                     const uint32_t a0 = smem_u32(st);
                     mbar_expect_tx(full, C::STAGE_BYTES);
-                    tma_load_2d(a0, &tm_act, kb * BK, act_row, full);
-                    tma_load_2d(a0 + C::A_BYTES, &tm_w1, kb * BK, w_row, full);
-                    if (SWIGLU) tma_load_2d(a0 + C::A_BYTES + 128 * 128, &tm_w2, kb * BK, w_row, full);
+                    if constexpr (!SWAP) {
+                        tma_load_2d(a0, &tm_act, kb * BK, act_row, full);
+                        tma_load_2d(a0 + C::A_BYTES, &tm_w1, kb * BK, w_row, full);
+                        if (SWIGLU) tma_load_2d(a0 + C::A_BYTES + 128 * 128, &tm_w2, kb * BK, w_row, full);
+                    } else {
+                        tma_load_2d(a0, &tm_w1, kb * BK, w_row, full);
+                        if (SWIGLU) tma_load_2d(a0 + C::A_BYTES, &tm_w2, kb * BK, w_row, full);
+                        tma_load_2d(a0 + C::NUM_A * C::A_BYTES, &tm_act, kb * BK, act_row, full);
+                    }
                 }
                 used |= 1u << stage;
                 last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
@@ -238,7 +259,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
-            const uint32_t idesc = idesc_bf16(128, C::MMA_N);
+            uint32_t idesc;
+            if constexpr (SWAP) {
+                int e, rb, cb;
+                decode_tile(aux, E, R, tile, e, rb, cb);
+                const int rows = min(R, aux.cnt[e] - rb * R);
+                idesc = idesc_bf16(128, (rows + 15) & ~15);
+            } else {
+                idesc = idesc_bf16(128, C::MMA_N);
+            }
             const uint32_t d_tmem = tmem_base + (uint32_t)(buf * C::ACC);
             bool ok = true;
             for (int kb = 0; kb < nk; ++kb) {
@@ -252,9 +281,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
                         const uint32_t acc = (kb | kk) ? 1u : 0u;
-                        // M = 128 A rows from the stage start: the RA staged token rows, then
-                        // bytes of the weight slice (rows never stored)
-                        tc_mma(d_tmem, sdesc_sw128(a0 + kk * 32), sdesc_sw128(a0 + C::A_BYTES + kk * 32), idesc, acc);
+                        if constexpr (!SWAP) {
+                            tc_mma(d_tmem, sdesc_sw128(a0 + kk * 32), sdesc_sw128(a0 + C::A_BYTES + kk * 32), idesc,
+                                   acc);
+                        } else {
+                            const uint32_t b0 = a0 + C::NUM_A * C::A_BYTES;
+                            tc_mma(d_tmem, sdesc_sw128(a0 + kk * 32), sdesc_sw128(b0 + kk * 32), idesc, acc);
+                            if (SWIGLU)
+                                tc_mma(d_tmem + R, sdesc_sw128(a0 + C::A_BYTES + kk * 32), sdesc_sw128(b0 + kk * 32),
+                                       idesc, acc);
+                        }
                     }
                     tc_commit(smem_u32(&aux.empty[stage]));
                 }
@@ -300,12 +336,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int rows = min(R, aux.cnt[e] - rb * R);
             const int64_t row0 = (int64_t)aux.off[e] + (int64_t)rb * R;
             const uint32_t tb = tmem_base + (uint32_t)(buf * C::ACC) + ((uint32_t)(32 * q) << 16);
-            const int m = 32 * q + lane;  // activation row inside the tile
-            if (32 * q < rows) {  // warp-uniform: lane quarters past the staged rows hold nothing to store
+            if constexpr (!SWAP) {
+                const int m = 32 * q + lane;  // activation row inside the tile
                 uint16_t* orow = p.out + (row0 + m) * p.ldo + (int64_t)cb * COLS;
                 const bool valid = m < rows;
+                // warp-uniform: a lane quarter past the tile's rows holds nothing to store
 #pragma unroll 1
-                for (int c = 0; c < COLS; c += 32) {
+                for (int c = 0; c < (32 * q < rows ? COLS : 0); c += 32) {
                     uint32_t g[32];
                     tmem_ld32(tb + c, g);
                     uint32_t pk[16];
@@ -328,6 +365,31 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int v = 0; v < 4; ++v)
                             st16(orow + c + 8 * v, make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]));
+                    }
+                }
+            } else {
+                const int f = 32 * q + lane;  // weight row (output column) inside the tile
+                uint16_t* ocol = p.out + row0 * p.ldo + (int64_t)cb * 128 + f;
+#pragma unroll 1
+                for (int c = 0; c < rows; c += C::LDW) {
+                    uint32_t g[C::LDW];
+                    tmem_ld(tb + c, g);
+                    if constexpr (SWIGLU) {
+                        uint32_t u[C::LDW];
+                        tmem_ld(tb + R + c, u);
+                        tmem_wait_ld(g);
+                        tmem_wait_ld(u);
+#pragma unroll
+                        for (int i = 0; i < C::LDW; ++i)
+                            if (c + i < rows)
+                                ocol[(int64_t)(c + i) * p.ldo] = (uint16_t)f32_to_bf16_bits(
+                                    silu_mul(__uint_as_float(g[i]), __uint_as_float(u[i])));
+                    } else {
+                        tmem_wait_ld(g);
+#pragma unroll
+                        for (int i = 0; i < C::LDW; ++i)
+                            if (c + i < rows)
+                                ocol[(int64_t)(c + i) * p.ldo] = (uint16_t)f32_to_bf16_bits(__uint_as_float(g[i]));
                     }
                 }
             }
@@ -359,10 +421,10 @@ static bool encode_2d(CUtensorMap* tm, const void* base, uint64_t inner, uint64_
     return r == CUDA_SUCCESS;
 }
 
-template <bool SWIGLU, int R, int COLS>
+template <bool SWAP, bool SWIGLU, int R, int COLS>
 static cudaError_t run(const Ctx& c, const void* act, int S, const void* w1, const void* w2, const Args& a) {
-    using C = Cfg<SWIGLU, R, COLS>;
-    auto kern = grouped_gemm_kernel<SWIGLU, R, COLS>;
+    using C = Cfg<SWAP, SWIGLU, R, COLS>;
+    auto kern = grouped_gemm_kernel<SWAP, SWIGLU, R, COLS>;
     static bool attr_done[64] = {};
     if (c.device < 0 || c.device >= 64) return cudaErrorInvalidDevice;
     if (!attr_done[c.device]) {
@@ -382,16 +444,25 @@ static cudaError_t run(const Ctx& c, const void* act, int S, const void* w1, con
     return launch(kern, dim3(grid), dim3(kThreads), (size_t)C::SMEM, c, tm_act, tm_w1, tm_w2, a);
 }
 
-// Token rows staged per tile: the smallest of 16/32/64/128 that holds about
-// three times the average rows per expert, so nearly every expert takes one
-// row block and reads each weight tile once.  The MMA is M = 128 either way;
-// a smaller block only saves shared memory and activation reads.
+// Token rows staged per rows-as-M tile: the smallest of 16/32/64/128 that
+// holds about three times the average rows per expert, so nearly every
+// expert takes one row block and reads each weight tile once.
 static int pick_rows(int S, int E) {
     const int64_t want = E > 0 ? 3 * ((int64_t)S + E - 1) / E : 0;
     if (want <= 16) return 16;
     if (want <= 32) return 32;
     if (want <= 64) return 64;
     return 128;
+}
+
+// Row block of the weights-as-M gate/up tile (about twice the average), or 0
+// when experts average more than 32 rows and rows-as-M is used.
+static int pick_swap_rows(int S, int E) {
+    const int avg = E > 0 ? S / E : 0;
+    if (avg <= 8) return 16;
+    if (avg <= 16) return 32;
+    if (avg <= 32) return 64;
+    return 0;
 }
 
 }  // namespace tc
@@ -401,12 +472,13 @@ cudaError_t launch_gate_up_bf16(const Ctx& c, const void* xp, const void* Wg, co
     if (S == 0) return cudaSuccess;
     if (use_pair_gemm(S, E, 256)) return launch_gate_up_bf16_pair(c, xp, Wg, Wu, counts, offsets, S, E, d, d_ff, h, status);
     tc::Args a{counts, offsets, E, d, d_ff, static_cast<uint16_t*>(h), (int64_t)d_ff, status};
-    switch (tc::pick_rows(S, E)) {
-        case 16: return tc::run<true, 16, 128>(c, xp, S, Wg, Wu, a);
-        case 32: return tc::run<true, 32, 128>(c, xp, S, Wg, Wu, a);
-        case 64: return tc::run<true, 64, 128>(c, xp, S, Wg, Wu, a);
-        default: return tc::run<true, 128, 128>(c, xp, S, Wg, Wu, a);
+    switch (tc::pick_swap_rows(S, E)) {
+        case 16: return tc::run<true, true, 16, 128>(c, xp, S, Wg, Wu, a);
+        case 32: return tc::run<true, true, 32, 128>(c, xp, S, Wg, Wu, a);
+        case 64: return tc::run<true, true, 64, 128>(c, xp, S, Wg, Wu, a);
+        default: break;
     }
+    return tc::run<false, true, 128, 128>(c, xp, S, Wg, Wu, a);  // above 32 rows per expert pick_rows() is 128
 }
 
 cudaError_t launch_down_bf16(const Ctx& c, const void* h, const void* Wd, const int32_t* counts, const int32_t* offsets,
@@ -417,17 +489,17 @@ cudaError_t launch_down_bf16(const Ctx& c, const void* h, const void* Wd, const 
     const int ra = tc::pick_rows(S, E);
     if (d % 256 == 0) {
         switch (ra) {
-            case 16: return tc::run<false, 16, 256>(c, h, S, Wd, nullptr, a);
-            case 32: return tc::run<false, 32, 256>(c, h, S, Wd, nullptr, a);
-            case 64: return tc::run<false, 64, 256>(c, h, S, Wd, nullptr, a);
-            default: return tc::run<false, 128, 256>(c, h, S, Wd, nullptr, a);
+            case 16: return tc::run<false, false, 16, 256>(c, h, S, Wd, nullptr, a);
+            case 32: return tc::run<false, false, 32, 256>(c, h, S, Wd, nullptr, a);
+            case 64: return tc::run<false, false, 64, 256>(c, h, S, Wd, nullptr, a);
+            default: return tc::run<false, false, 128, 256>(c, h, S, Wd, nullptr, a);
         }
     }
     switch (ra) {
-        case 16: return tc::run<false, 16, 128>(c, h, S, Wd, nullptr, a);
-        case 32: return tc::run<false, 32, 128>(c, h, S, Wd, nullptr, a);
-        case 64: return tc::run<false, 64, 128>(c, h, S, Wd, nullptr, a);
-        default: return tc::run<false, 128, 128>(c, h, S, Wd, nullptr, a);
+        case 16: return tc::run<false, false, 16, 128>(c, h, S, Wd, nullptr, a);
+        case 32: return tc::run<false, false, 32, 128>(c, h, S, Wd, nullptr, a);
+        case 64: return tc::run<false, false, 64, 128>(c, h, S, Wd, nullptr, a);
+        default: return tc::run<false, false, 128, 128>(c, h, S, Wd, nullptr, a);
     }
 }
 
