@@ -66,13 +66,18 @@ def build(force: bool = False, ptxas_v: bool = False, verbose: bool = False) -> 
         for _, log in results:
             if log:
                 sys.stderr.write(log)
-    if force or _stale(LIB, objs):
+    # the object list of the last link: a source that was removed must leave the library too
+    manifest = os.path.join(OUT_DIR, "link_objects.txt")
+    listed = open(manifest).read().split() if os.path.exists(manifest) else []
+    if force or _stale(LIB, objs) or sorted(listed) != sorted(objs):
         tmp = LIB + f".tmp{os.getpid()}"
         cmd = [NVCC, *ARCH, "-shared", "-o", tmp, *objs]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"nvcc link failed:\n{r.stdout}\n{r.stderr}")
         os.replace(tmp, LIB)
+        with open(manifest, "w") as f:
+            f.write("\n".join(objs) + "\n")
     return LIB
 
 
