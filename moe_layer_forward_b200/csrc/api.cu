@@ -282,7 +282,10 @@ moe_status_t moe_forward(const moe_shape_t* shape, const moe_weights_t* wts, con
     int32_t* offsets = static_cast<int32_t*>(cv.take((size_t)(E + 1) * sizeof(int32_t)));
     int32_t* slot_token = static_cast<int32_t*>(cv.take((size_t)S * sizeof(int32_t)));
     int32_t* token_slot = static_cast<int32_t*>(cv.take((size_t)S * sizeof(int32_t)));
-    void* xp = cv.take((size_t)S * d * es);
+    // bf16 experts on one-CTA tiles read their rows straight from v through slot_token; only the
+    // fp32 path and the CTA-pair tiles need the permuted copy Xp
+    const bool fused_gather = wdt == MOE_BF16 && !gate_up_needs_permuted_rows(S, E);
+    void* xp = fused_gather ? nullptr : cv.take((size_t)S * d * es);
     void* h = cv.take((size_t)S * d_ff * es);
     void* y = cv.take((size_t)S * d * es);
     bool query = false;
@@ -317,8 +320,8 @@ moe_status_t moe_forward(const moe_shape_t* shape, const moe_weights_t* wts, con
     if (st != MOE_OK) return st;
     // 4. grouped SwiGLU MLP
     if (wdt == MOE_BF16) {
-        st = cuda_status(launch_gate_up_bf16(c, xp, wts->W_gate, wts->W_up, counts, offsets, S, E, d, d_ff, h,
-                                             dev_status));
+        st = cuda_status(launch_gate_up_bf16(c, fused_gather ? v : xp, wts->W_gate, wts->W_up, counts, offsets, S, E,
+                                             d, d_ff, h, dev_status, fused_gather ? slot_token : nullptr, T));
         if (st != MOE_OK) return st;
         st = cuda_status(launch_down_bf16(c, h, wts->W_down, counts, offsets, S, E, d, d_ff, y, dev_status));
     } else {

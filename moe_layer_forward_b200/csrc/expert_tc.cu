@@ -56,7 +56,9 @@ namespace moe {
 namespace tc {
 
 constexpr int BK = 64;  // K elements per stage = one 128-byte swizzle row of bf16
-constexpr int kThreads = 192;
+// warps 0..5 as below; the weights-as-M form adds warps 6..9 that gather activation rows (Args::gather)
+template <bool SWAP>
+constexpr int threads_of() { return SWAP ? 320 : 192; }
 constexpr int kSmemLimit = 232448;              // 227 KB opt-in per CTA
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
@@ -75,6 +77,9 @@ struct Cfg {
     static constexpr int A_BYTES = A_ROWS * 128;
     static constexpr int B_BYTES = B_ROWS * 128;
     static constexpr int STAGE_BYTES = NUM_A * A_BYTES + B_BYTES;
+    // the activation slice of a stage: A for rows-as-M, B for weights-as-M
+    static constexpr int ACT_OFF = SWAP ? NUM_A * A_BYTES : 0;
+    static constexpr int ACT_BYTES = R * 128;
     // rows-as-M reads 128 A rows from the stage start: they must stay inside the stage
     static_assert(SWAP || STAGE_BYTES >= 128 * 128, "M = 128 operand inside its stage");
     static constexpr int WBOX = SWAP ? 128 : (SWIGLU ? 128 : COLS);  // weight rows per TMA box
@@ -99,7 +104,17 @@ struct Args {
     uint16_t* out;
     int64_t ldo;
     int32_t* status;
+    // Optional row gather: when set, activation row i of the expert-contiguous
+    // order is row gather[i] of act (the permutation's slot -> token map), read
+    // by the gather warps instead of a TMA load of a permuted copy.
+    const int32_t* gather;
+    const uint16_t* act;
 };
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 struct Aux {  // lives after the stage ring in shared memory
     uint64_t full[12];
@@ -128,7 +143,7 @@ __device__ __forceinline__ void decode_tile(const Aux& a, int E, int R, int tile
 }
 
 template <bool SWAP, bool SWIGLU, int R, int COLS>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(threads_of<SWAP>(), 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_w1,
                         const __grid_constant__ CUtensorMap tm_w2, const Args p) {
     using C = Cfg<SWAP, SWIGLU, R, COLS>;
@@ -142,7 +157,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- prologue (overlaps the previous kernel's tail under PDL)
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(smem_u32(&aux.full[s]), 1);
+            mbar_init(smem_u32(&aux.full[s]), p.gather ? 2 : 1);  // + the gather warp's arrival
             mbar_init(smem_u32(&aux.empty[s]), 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -160,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     pdl_wait();
     const int E = p.E;
-    for (int e = threadIdx.x; e < E; e += kThreads) {
+    for (int e = threadIdx.x; e < E; e += (int)blockDim.x) {
         aux.cnt[e] = p.counts[e];
         aux.off[e] = p.offsets[e];
     }
@@ -220,15 +235,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) {
                     uint8_t* st = smem + stage * C::STAGE_BYTES;
                     const uint32_t a0 = smem_u32(st);
-                    mbar_expect_tx(full, C::STAGE_BYTES);
+                    const bool gath = p.gather != nullptr;
+                    mbar_expect_tx(full, C::STAGE_BYTES - (gath ? C::ACT_BYTES : 0));
                     if constexpr (!SWAP) {
-                        tma_load_2d(a0, &tm_act, kb * BK, act_row, full);
+                        if (!gath) tma_load_2d(a0, &tm_act, kb * BK, act_row, full);
                         tma_load_2d(a0 + C::A_BYTES, &tm_w1, kb * BK, w_row, full);
                         if (SWIGLU) tma_load_2d(a0 + C::A_BYTES + 128 * 128, &tm_w2, kb * BK, w_row, full);
                     } else {
                         tma_load_2d(a0, &tm_w1, kb * BK, w_row, full);
                         if (SWIGLU) tma_load_2d(a0 + C::A_BYTES, &tm_w2, kb * BK, w_row, full);
-                        tma_load_2d(a0 + C::NUM_A * C::A_BYTES, &tm_act, kb * BK, act_row, full);
+                        if (!gath) tma_load_2d(a0 + C::NUM_A * C::A_BYTES, &tm_act, kb * BK, act_row, full);
                     }
                 }
                 used |= 1u << stage;
@@ -316,6 +332,58 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait(smem_u32(&aux.drain), 0, abort_flag);
         }
         __syncwarp();
+    } else if (SWAP && warp >= 6) {
+        // ================= row gather (warps 6..9, only with p.gather): warp gw fills the stages
+        // g = gw, gw + 4, ... with the tile's activation rows, 16-byte cp.async chunks into the
+        // 128-byte-swizzled layout a TMA load would produce (chunk c of row r at r*128 + (c ^ r%8)*16).
+        // It waits for its own copies and fences them into the async proxy before arriving on the
+        // stage's full barrier, which the tensor cores' reads are ordered after.
+        if (p.gather != nullptr) {  // weights-as-M only: the rows are the B operand, R <= 64
+            constexpr int RPL = R / 4;    // rows per lane: lane covers rows (lane / 8) + 4 i
+            const int gw = warp - 6;
+            const int nk = p.K / BK;
+            const int c = lane & 7, r0 = lane >> 3;
+            int tok[RPL];
+            int cur = -1, rows = 0;
+            for (int g = gw;; g += 4) {
+                const int ti = g / nk, kb = g - ti * nk;
+                const int tile = blockIdx.x + ti * gridDim.x;
+                if (tile >= total || *abort_flag) break;
+                if (tile != cur) {
+                    int e, rb, cb;
+                    decode_tile(aux, E, R, tile, e, rb, cb);
+                    rows = min(R, aux.cnt[e] - rb * R);
+                    const int base = aux.off[e] + rb * R;
+#pragma unroll
+                    for (int i = 0; i < RPL; ++i) {
+                        const int r = r0 + 4 * i;
+                        tok[i] = r < rows ? p.gather[base + r] : 0;
+                    }
+                    cur = tile;
+                }
+                const int stage = g % STAGES;
+                const uint32_t use = (uint32_t)(g / STAGES);
+                if (!warp_wait(smem_u32(&aux.empty[stage]), (use & 1u) ^ 1u, abort_flag)) {
+                    if (lane == 0) {
+                        *abort_flag = 1;
+                        set_status(p.status, DEV_TIMEOUT);
+                    }
+                    break;
+                }
+                const uint32_t dst = smem_u32(smem + stage * C::STAGE_BYTES) + C::ACT_OFF;
+                const uint16_t* src = p.act + (int64_t)kb * BK + c * 8;
+#pragma unroll
+                for (int i = 0; i < RPL; ++i) {
+                    const int r = r0 + 4 * i;
+                    if (r < rows)  // rows past the tile's count feed only accumulator entries that are never stored
+                        cp_async16(dst + r * 128 + ((c ^ (r & 7)) << 4), src + (int64_t)tok[i] * p.K);
+                }
+                cp_async_wait_all();
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&aux.full[stage]));
+            }
+        }
     } else {
         // ================= epilogue (warps 2..5 -> TMEM lane quarters 2,3,0,1)
         const int q = warp & 3;
@@ -422,7 +490,8 @@ static bool encode_2d(CUtensorMap* tm, const void* base, uint64_t inner, uint64_
 }
 
 template <bool SWAP, bool SWIGLU, int R, int COLS>
-static cudaError_t run(const Ctx& c, const void* act, int S, const void* w1, const void* w2, const Args& a) {
+static cudaError_t run(const Ctx& c, const void* act, int S, const void* w1, const void* w2, const Args& a,
+                       int act_rows = -1) {
     using C = Cfg<SWAP, SWIGLU, R, COLS>;
     auto kern = grouped_gemm_kernel<SWAP, SWIGLU, R, COLS>;
     static bool attr_done[64] = {};
@@ -433,7 +502,10 @@ static cudaError_t run(const Ctx& c, const void* act, int S, const void* w1, con
         attr_done[c.device] = true;
     }
     CUtensorMap tm_act, tm_w1, tm_w2;
-    if (!encode_2d(&tm_act, act, (uint64_t)a.K, (uint64_t)S, (uint32_t)R)) return cudaErrorInvalidValue;
+    // act holds S permuted rows, or (with a.gather) act_rows rows read through the slot -> row map
+    const uint64_t arows = act_rows >= 0 ? (uint64_t)act_rows : (uint64_t)S;
+    if (arows == 0) return cudaErrorInvalidValue;
+    if (!encode_2d(&tm_act, act, (uint64_t)a.K, arows, (uint32_t)R)) return cudaErrorInvalidValue;
     if (!encode_2d(&tm_w1, w1, (uint64_t)a.K, (uint64_t)a.E * a.n_out, (uint32_t)C::WBOX)) return cudaErrorInvalidValue;
     if (!encode_2d(&tm_w2, SWIGLU ? w2 : w1, (uint64_t)a.K, (uint64_t)a.E * a.n_out, (uint32_t)C::WBOX))
         return cudaErrorInvalidValue;
@@ -441,7 +513,7 @@ static cudaError_t run(const Ctx& c, const void* act, int S, const void* w1, con
     const int64_t max_tiles = ((int64_t)S / R + a.E) * (a.n_out / COLS);
     const int grid = (int)(max_tiles < c.num_sms ? max_tiles : c.num_sms);
     if (grid <= 0) return cudaSuccess;
-    return launch(kern, dim3(grid), dim3(kThreads), (size_t)C::SMEM, c, tm_act, tm_w1, tm_w2, a);
+    return launch(kern, dim3(grid), dim3(threads_of<SWAP>()), (size_t)C::SMEM, c, tm_act, tm_w1, tm_w2, a);
 }
 
 // Token rows staged per rows-as-M tile: the smallest of 16/32/64/128 that
@@ -467,25 +539,35 @@ static int pick_swap_rows(int S, int E) {
 
 }  // namespace tc
 
+// Only the weights-as-M gate/up form (few rows per expert) gathers its rows in place: there a tile
+// stages at most 64 rows per K slice, which four gather warps copy well within a stage's time.  For
+// 128-row tiles the gather warps could not keep the ring full (measured: prefill 11% slower than
+// copying the rows once with the permutation), so those read the permuted copy by TMA.
+bool gate_up_needs_permuted_rows(int S, int E) { return use_pair_gemm(S, E, 256) || tc::pick_swap_rows(S, E) == 0; }
+
 cudaError_t launch_gate_up_bf16(const Ctx& c, const void* xp, const void* Wg, const void* Wu, const int32_t* counts,
-                                const int32_t* offsets, int S, int E, int d, int d_ff, void* h, int32_t* status) {
+                                const int32_t* offsets, int S, int E, int d, int d_ff, void* h, int32_t* status,
+                                const int32_t* gather, int act_rows) {
     if (S == 0) return cudaSuccess;
+    if (gather && gate_up_needs_permuted_rows(S, E)) return cudaErrorInvalidValue;
     if (use_pair_gemm(S, E, 256)) return launch_gate_up_bf16_pair(c, xp, Wg, Wu, counts, offsets, S, E, d, d_ff, h, status);
-    tc::Args a{counts, offsets, E, d, d_ff, static_cast<uint16_t*>(h), (int64_t)d_ff, status};
+    tc::Args a{counts, offsets, E, d, d_ff, static_cast<uint16_t*>(h), (int64_t)d_ff, status, gather,
+               static_cast<const uint16_t*>(xp)};
+    const int ar = gather ? act_rows : -1;
     switch (tc::pick_swap_rows(S, E)) {
-        case 16: return tc::run<true, true, 16, 128>(c, xp, S, Wg, Wu, a);
-        case 32: return tc::run<true, true, 32, 128>(c, xp, S, Wg, Wu, a);
-        case 64: return tc::run<true, true, 64, 128>(c, xp, S, Wg, Wu, a);
+        case 16: return tc::run<true, true, 16, 128>(c, xp, S, Wg, Wu, a, ar);
+        case 32: return tc::run<true, true, 32, 128>(c, xp, S, Wg, Wu, a, ar);
+        case 64: return tc::run<true, true, 64, 128>(c, xp, S, Wg, Wu, a, ar);
         default: break;
     }
-    return tc::run<false, true, 128, 128>(c, xp, S, Wg, Wu, a);  // above 32 rows per expert pick_rows() is 128
+    return tc::run<false, true, 128, 128>(c, xp, S, Wg, Wu, a, ar);  // above 32 rows per expert pick_rows() is 128
 }
 
 cudaError_t launch_down_bf16(const Ctx& c, const void* h, const void* Wd, const int32_t* counts, const int32_t* offsets,
                              int S, int E, int d, int d_ff, void* y, int32_t* status) {
     if (S == 0) return cudaSuccess;
     if (use_pair_gemm(S, E, d)) return launch_down_bf16_pair(c, h, Wd, counts, offsets, S, E, d, d_ff, y, status);
-    tc::Args a{counts, offsets, E, d_ff, d, static_cast<uint16_t*>(y), (int64_t)d, status};
+    tc::Args a{counts, offsets, E, d_ff, d, static_cast<uint16_t*>(y), (int64_t)d, status, nullptr, nullptr};
     const int ra = tc::pick_rows(S, E);
     if (d % 256 == 0) {
         switch (ra) {

@@ -65,13 +65,19 @@ inline size_t permute_ws_bytes(int T, int E) {
     size_t nchunks = (size_t)(T + kPermuteChunk - 1) / kPermuteChunk;
     return nchunks * (size_t)E * sizeof(int32_t);
 }
+// xp == nullptr: only the maps (counts, offsets, slot_token, token_slot), no row copy
 cudaError_t launch_permute(const Ctx& c, const void* v, int v_dt, const int32_t* idx, int T, int d, int E, int k,
                            int32_t* counts, int32_t* offsets, int32_t* slot_token, int32_t* token_slot, void* xp,
                            int32_t* hist, int32_t* status);
 
 // ---- step 4: expert MLP (expert_tc.cu: bf16 tensor cores; expert_simt.cu: fp32)
+// gate/up: xp holds the S permuted rows; or, with gather, xp holds act_rows rows and slot i
+// reads row gather[i] (the permutation's slot -> token map), so no permuted copy is made.
+// The CTA-pair kernel needs the permuted copy (gate_up_needs_permuted_rows()).
+bool gate_up_needs_permuted_rows(int S, int E);
 cudaError_t launch_gate_up_bf16(const Ctx& c, const void* xp, const void* Wg, const void* Wu, const int32_t* counts,
-                                const int32_t* offsets, int S, int E, int d, int d_ff, void* h, int32_t* status);
+                                const int32_t* offsets, int S, int E, int d, int d_ff, void* h, int32_t* status,
+                                const int32_t* gather = nullptr, int act_rows = 0);
 cudaError_t launch_down_bf16(const Ctx& c, const void* h, const void* Wd, const int32_t* counts, const int32_t* offsets,
                              int S, int E, int d, int d_ff, void* y, int32_t* status);
 // CTA-pair (cta_group::2) variants for experts with many rows each (expert_tc2.cu)

@@ -158,7 +158,7 @@ cudaError_t launch_permute(const Ctx& c, const void* v, int v_dt, const int32_t*
     if (err != cudaSuccess || T == 0) return err;
     err = launch(perm_scatter_kernel, dim3(nchunks), dim3(PC), 0, c, idx, T, E, k, hist, offsets, slot_token,
                  token_slot);
-    if (err != cudaSuccess) return err;
+    if (err != cudaSuccess || xp == nullptr) return err;
     const int64_t row_bytes = (int64_t)d * (v_dt == DT_BF16 ? 2 : 4);
     const int64_t n = (int64_t)T * (row_bytes / 16);
     int64_t blocks = (n + 255) / 256;
