@@ -20,6 +20,8 @@
 //                        order, scores sigmoid(z)+b in fp32 (sigmoid in double,
 //                        rounded once), then k rounds of a warp-shuffle argmax
 //                        (ties to the lower index) plus one more for the margin.
+//   router_topk_token_kernel  the same for few tokens: a CTA per token, a thread
+//                        per expert for the split sum, then one warp selects.
 #include <math.h>
 
 #include "common.cuh"
@@ -117,29 +119,14 @@ cudaError_t launch_rmsnorm(const Ctx& c, const void* x, int x_dt, const float* g
 // ----------------------------------------------------------------------------- top-k
 __device__ __forceinline__ bool better(float ka, int ea, float kb, int eb) { return ka > kb || (ka == kb && ea < eb); }
 
-__global__ void __launch_bounds__(256) router_topk_kernel(const float* __restrict__ partial, int splitk,
-                                                          const float* __restrict__ b, int T, int E, int k,
-                                                          int32_t* __restrict__ idx, float* __restrict__ w,
-                                                          float* __restrict__ logits, float* __restrict__ margin) {
-    pdl_wait();
-    pdl_trigger();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t = blockIdx.x * 8 + warp;
-    if (t >= T) return;
-    float z[8], key[8];
+// Scores, top-k selection and weights of token t from its logits z[j] = z(lane + 32 j), by one
+// warp: sigmoid in double rounded once to fp32, + b in fp32, k rounds of a warp-shuffle argmax
+// (ties to the lower index) and one more for the margin to the first expert left out.
+__device__ __forceinline__ void select_topk_warp(const float (&z)[8], int lane, int t, const float* __restrict__ b,
+                                                 int E, int k, int32_t* __restrict__ idx, float* __restrict__ w,
+                                                 float* __restrict__ logits, float* __restrict__ margin) {
+    float key[8];
     uint32_t taken = 0;  // bit j: entry lane + 32 j unavailable
-#pragma unroll
-    for (int j = 0; j < 8; ++j) z[j] = 0.f;
-    // sum the K-split partials in split order; the loads of one split are independent of each other
-#pragma unroll 4
-    for (int s = 0; s < splitk; ++s) {
-        const float* ps = partial + ((int64_t)s * T + t) * E;
-        float pv[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) pv[j] = (lane + 32 * j < E) ? __ldg(ps + lane + 32 * j) : 0.f;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) z[j] += pv[j];
-    }
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         const int e = lane + 32 * j;
@@ -211,9 +198,68 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
     if (margin && lane == 0) margin[t] = (E > k) ? (kth - next) : INFINITY;
 }
 
+__global__ void __launch_bounds__(256) router_topk_kernel(const float* __restrict__ partial, int splitk,
+                                                          const float* __restrict__ b, int T, int E, int k,
+                                                          int32_t* __restrict__ idx, float* __restrict__ w,
+                                                          float* __restrict__ logits, float* __restrict__ margin) {
+    pdl_wait();
+    pdl_trigger();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = blockIdx.x * 8 + warp;
+    if (t >= T) return;
+    float z[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) z[j] = 0.f;
+    // sum the K-split partials in split order; the loads of one split are independent of each other
+#pragma unroll 4
+    for (int s = 0; s < splitk; ++s) {
+        const float* ps = partial + ((int64_t)s * T + t) * E;
+        float pv[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) pv[j] = (lane + 32 * j < E) ? __ldg(ps + lane + 32 * j) : 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) z[j] += pv[j];
+    }
+    select_topk_warp(z, lane, t, b, E, k, idx, w, logits, margin);
+}
+
+// Few tokens (decode): one CTA per token, one thread per expert, so the split partials of all
+// experts load in parallel (each thread's own sum still runs in split order: the same logits as
+// the warp-per-token kernel bit for bit); then warp 0 selects.
+__global__ void __launch_bounds__(256) router_topk_token_kernel(const float* __restrict__ partial, int splitk,
+                                                                const float* __restrict__ b, int T, int E, int k,
+                                                                int32_t* __restrict__ idx, float* __restrict__ w,
+                                                                float* __restrict__ logits,
+                                                                float* __restrict__ margin) {
+    __shared__ float zs[kMaxExperts];
+    pdl_wait();
+    pdl_trigger();
+    const int t = blockIdx.x, e = threadIdx.x;
+    if (e < E) {
+        const float* pe = partial + (int64_t)t * E + e;
+        const int64_t stride = (int64_t)T * E;
+        float acc = 0.f;
+#pragma unroll 8
+        for (int s = 0; s < splitk; ++s) acc += __ldg(pe + s * stride);
+        zs[e] = acc;
+    }
+    __syncthreads();
+    if (threadIdx.x >= 32) return;
+    const int lane = threadIdx.x;
+    float z[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) z[j] = (lane + 32 * j < E) ? zs[lane + 32 * j] : 0.f;
+    select_topk_warp(z, lane, t, b, E, k, idx, w, logits, margin);
+}
+
 cudaError_t launch_router_topk(const Ctx& c, const RouterPlan& p, const float* partial, const float* b, int T, int E,
                                int k, int32_t* idx, float* w, float* logits, float* margin) {
     if (T == 0) return cudaSuccess;
+    if (T <= c.num_sms && p.splitk > 2) {  // a warp per token would occupy only T / 8 SMs
+        const int threads = (E + 31) / 32 * 32;
+        return launch(router_topk_token_kernel, dim3(T), dim3(threads < 32 ? 32 : threads), 0, c, partial, p.splitk,
+                      b, T, E, k, idx, w, logits, margin);
+    }
     return launch(router_topk_kernel, dim3((T + 7) / 8), dim3(256), 0, c, partial, p.splitk, b, T, E, k, idx, w,
                   logits, margin);
 }
