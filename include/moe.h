@@ -56,6 +56,7 @@ typedef enum {
 /* bits OR-ed into *dev_status by kernels */
 #define MOE_DEV_BAD_EXPERT_ID 1 /* topk_idx held an id outside [0, E); that pair was dropped */
 #define MOE_DEV_TIMEOUT 2       /* a bounded in-kernel wait gave up; outputs are not valid */
+#define MOE_DEV_BAD_COUNT 4     /* a masked-layout count was outside [0, cap]; it was clamped */
 
 #define MOE_MAX_EXPERTS 256
 #define MOE_MAX_TOP_K 8
@@ -180,6 +181,28 @@ moe_status_t moe_expert_down(const void* h, const void* W_down, moe_dtype_t dt, 
 moe_status_t moe_grouped_swiglu(const void* xp, const void* W_gate, const void* W_up, const void* W_down,
                                 moe_dtype_t dt, const int32_t* counts, const int32_t* offsets, int32_t S, int32_t E,
                                 int32_t d, int32_t d_ff, void* h, void* y, int32_t* dev_status, moe_stream_t stream);
+
+/*
+ * Step 4 on the masked decode layout [P5 §专家计算实现: deepgemm_masked, the
+ * decode-phase expert GEMM; the page names it without defining it, and this
+ * follows the reading that its input is per-expert buffers of fixed capacity
+ * with a valid-row count per expert, the form a low-latency token dispatch
+ * writes]:
+ *   for every expert e and row r < counts[e]:
+ *     h[e][r][f] = SiLU(x[e][r] . W_gate[e][f]) * (x[e][r] . W_up[e][f])
+ *     y[e][r][o] = h[e][r] . W_down[e][o]
+ * x [E][cap][d], h [E][cap][d_ff], y [E][cap][d]; counts [E] on the device.
+ * Rows r >= counts[e] are neither used for any stored result nor written, so
+ * the buffers need no clearing and the call never reads counts on the host
+ * (its launch configuration depends on E, cap, d, d_ff only, so one capture
+ * into a CUDA graph serves any counts).  A count outside [0, cap] is clamped
+ * and sets MOE_DEV_BAD_COUNT.  Same kernels and numerics as moe_grouped_swiglu
+ * (one-CTA tiles); dt must be MOE_BF16; 1 <= cap, E * cap < 2^30; d % 128 == 0,
+ * d_ff % 128 == 0; 16-byte aligned pointers.
+ */
+moe_status_t moe_grouped_swiglu_masked(const void* x, const void* W_gate, const void* W_up, const void* W_down,
+                                       moe_dtype_t dt, const int32_t* counts, int32_t E, int32_t cap, int32_t d,
+                                       int32_t d_ff, void* h, void* y, int32_t* dev_status, moe_stream_t stream);
 
 /*
  * Step 5 — weighted un-permute and residual [P1 §EP 路径: weighted sum at the

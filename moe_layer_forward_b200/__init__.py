@@ -47,6 +47,7 @@ _sig = {
     "moe_expert_gate_up": [_vp, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp],
     "moe_expert_down": [_vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp],
     "moe_grouped_swiglu": [_vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp],
+    "moe_grouped_swiglu_masked": [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp],
     "moe_unpermute_combine": [_vp, _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _i32, _vp],
     "moe_forward": [ctypes.POINTER(MoeShape), ctypes.POINTER(MoeWeights), _vp, _vp, _vp, _vp, _vp, _vp, _szp, _vp,
                     _vp],
@@ -178,6 +179,15 @@ def moe_grouped_swiglu(xp, W_gate, W_up, W_down, counts, offsets, h, y, dev_stat
     _check("moe_grouped_swiglu", _lib.moe_grouped_swiglu(_p(xp), _p(W_gate), _p(W_up), _p(W_down), _dt(W_gate),
                                                          _p(counts), _p(offsets), S, E, d, d_ff, _p(h), _p(y),
                                                          _p(dev_status), _stream(xp.device)))
+
+
+def moe_grouped_swiglu_masked(x, W_gate, W_up, W_down, counts, h, y, dev_status=None) -> None:
+    """Expert MLP on per-expert buffers x [E][cap][d] with counts [E] valid rows each (device)."""
+    E, cap, d = x.shape
+    d_ff = W_gate.shape[1]
+    _check("moe_grouped_swiglu_masked",
+           _lib.moe_grouped_swiglu_masked(_p(x), _p(W_gate), _p(W_up), _p(W_down), _dt(W_gate), _p(counts), E, cap,
+                                          d, d_ff, _p(h), _p(y), _p(dev_status), _stream(x.device)))
 
 
 def moe_unpermute_combine(y, token_slot, topk_w, residual, out) -> None:

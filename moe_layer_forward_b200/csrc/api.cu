@@ -231,6 +231,27 @@ moe_status_t moe_grouped_swiglu(const void* xp, const void* W_gate, const void* 
     return moe_expert_down(h, W_down, dt, counts, offsets, S, E, d, d_ff, y, dev_status, stream);
 }
 
+moe_status_t moe_grouped_swiglu_masked(const void* x, const void* W_gate, const void* W_up, const void* W_down,
+                                       moe_dtype_t dt, const int32_t* counts, int32_t E, int32_t cap, int32_t d,
+                                       int32_t d_ff, void* h, void* y, int32_t* dev_status, moe_stream_t stream) {
+    if (cap <= 0 || E <= 0 || (int64_t)E * cap >= (int64_t(1) << 30)) return MOE_ERR_INVALID_ARG;
+    const int S = E * cap;
+    moe_status_t st = check_expert_shape(dt, S, E, d, d_ff);
+    if (st != MOE_OK) return st;
+    if (dt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (!x || !W_gate || !W_up || !W_down || !counts || !h || !y) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(W_gate) || !aligned16(W_up) || !aligned16(W_down) || !aligned16(h) ||
+        !aligned16(y))
+        return MOE_ERR_INVALID_ARG;
+    Ctx c;
+    st = make_ctx(stream, c);
+    if (st != MOE_OK) return st;
+    st = cuda_status(launch_gate_up_bf16(c, x, W_gate, W_up, counts, nullptr, S, E, d, d_ff, h, dev_status, nullptr, 0,
+                                         cap));
+    if (st != MOE_OK) return st;
+    return cuda_status(launch_down_bf16(c, h, W_down, counts, nullptr, S, E, d, d_ff, y, dev_status, cap));
+}
+
 moe_status_t moe_unpermute_combine(const void* y, moe_dtype_t y_dt, const int32_t* token_slot, const float* topk_w,
                                    const void* residual, moe_dtype_t r_dt, int32_t T, int32_t d, int32_t k, void* out,
                                    moe_dtype_t out_dt, moe_stream_t stream) {

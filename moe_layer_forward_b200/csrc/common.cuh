@@ -8,7 +8,7 @@
 namespace moe {
 
 enum : int { DT_F32 = 0, DT_BF16 = 1 };
-enum : int { DEV_BAD_EXPERT_ID = 1, DEV_TIMEOUT = 2 };
+enum : int { DEV_BAD_EXPERT_ID = 1, DEV_TIMEOUT = 2, DEV_BAD_COUNT = 4 };
 
 constexpr int kMaxExperts = 256;
 constexpr int kMaxTopK = 8;

@@ -109,6 +109,9 @@ struct Args {
     // by the gather warps instead of a TMA load of a permuted copy.
     const int32_t* gather;
     const uint16_t* act;
+    // Masked layout (cap > 0): expert e's rows are rows [e*cap, e*cap + counts[e]) of fixed
+    // per-expert buffers, offsets is unused, and a count outside [0, cap] is clamped and flagged.
+    int cap;
 };
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
@@ -176,8 +179,15 @@ __global__ void __launch_bounds__(threads_of<SWAP>(), 1)
     pdl_wait();
     const int E = p.E;
     for (int e = threadIdx.x; e < E; e += (int)blockDim.x) {
-        aux.cnt[e] = p.counts[e];
-        aux.off[e] = p.offsets[e];
+        if (p.cap > 0) {
+            const int n = p.counts[e];
+            if (n < 0 || n > p.cap) set_status(p.status, DEV_BAD_COUNT);
+            aux.cnt[e] = n < 0 ? 0 : (n > p.cap ? p.cap : n);
+            aux.off[e] = e * p.cap;
+        } else {
+            aux.cnt[e] = p.counts[e];
+            aux.off[e] = p.offsets[e];
+        }
     }
     __syncthreads();
     if (warp == 0) {
@@ -547,12 +557,13 @@ bool gate_up_needs_permuted_rows(int S, int E) { return use_pair_gemm(S, E, 256)
 
 cudaError_t launch_gate_up_bf16(const Ctx& c, const void* xp, const void* Wg, const void* Wu, const int32_t* counts,
                                 const int32_t* offsets, int S, int E, int d, int d_ff, void* h, int32_t* status,
-                                const int32_t* gather, int act_rows) {
+                                const int32_t* gather, int act_rows, int cap) {
     if (S == 0) return cudaSuccess;
-    if (gather && gate_up_needs_permuted_rows(S, E)) return cudaErrorInvalidValue;
-    if (use_pair_gemm(S, E, 256)) return launch_gate_up_bf16_pair(c, xp, Wg, Wu, counts, offsets, S, E, d, d_ff, h, status);
+    if (gather && (cap > 0 || gate_up_needs_permuted_rows(S, E))) return cudaErrorInvalidValue;
+    if (cap == 0 && use_pair_gemm(S, E, 256))
+        return launch_gate_up_bf16_pair(c, xp, Wg, Wu, counts, offsets, S, E, d, d_ff, h, status);
     tc::Args a{counts, offsets, E, d, d_ff, static_cast<uint16_t*>(h), (int64_t)d_ff, status, gather,
-               static_cast<const uint16_t*>(xp)};
+               static_cast<const uint16_t*>(xp), cap};
     const int ar = gather ? act_rows : -1;
     switch (tc::pick_swap_rows(S, E)) {
         case 16: return tc::run<true, true, 16, 128>(c, xp, S, Wg, Wu, a, ar);
@@ -564,10 +575,11 @@ cudaError_t launch_gate_up_bf16(const Ctx& c, const void* xp, const void* Wg, co
 }
 
 cudaError_t launch_down_bf16(const Ctx& c, const void* h, const void* Wd, const int32_t* counts, const int32_t* offsets,
-                             int S, int E, int d, int d_ff, void* y, int32_t* status) {
+                             int S, int E, int d, int d_ff, void* y, int32_t* status, int cap) {
     if (S == 0) return cudaSuccess;
-    if (use_pair_gemm(S, E, d)) return launch_down_bf16_pair(c, h, Wd, counts, offsets, S, E, d, d_ff, y, status);
-    tc::Args a{counts, offsets, E, d_ff, d, static_cast<uint16_t*>(y), (int64_t)d, status, nullptr, nullptr};
+    if (cap == 0 && use_pair_gemm(S, E, d))
+        return launch_down_bf16_pair(c, h, Wd, counts, offsets, S, E, d, d_ff, y, status);
+    tc::Args a{counts, offsets, E, d_ff, d, static_cast<uint16_t*>(y), (int64_t)d, status, nullptr, nullptr, cap};
     const int ra = tc::pick_rows(S, E);
     if (d % 256 == 0) {
         switch (ra) {

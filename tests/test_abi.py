@@ -137,6 +137,14 @@ def test_expert_and_combine_reject_bad_shapes_on_host(lib):
     assert g(_p(), _p(), _p(), 0, _p(), _p(), 64, 8, 12, 256, _p(), NULL, NULL) == UNSUPPORTED  # f32 needs d % 8
     assert g(_p(), _p(), _p(), 1, _p(), _p(), 0, 8, 128, 256, _p(), NULL, NULL) == OK  # no rows: nothing to do
     assert g(NULL, _p(), _p(), 1, _p(), _p(), 64, 8, 128, 256, _p(), NULL, NULL) == INVALID
+    m = lib.moe_grouped_swiglu_masked
+    m.argtypes = [V, V, V, V, ctypes.c_int, V, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, V, V,
+                  V, V]
+    assert m(_p(), _p(), _p(), _p(), 1, _p(), 8, 0, 128, 256, _p(), _p(), NULL, NULL) == INVALID  # cap >= 1
+    assert m(_p(), _p(), _p(), _p(), 1, _p(), 8, 1 << 28, 128, 256, _p(), _p(), NULL, NULL) == INVALID  # E*cap
+    assert m(_p(), _p(), _p(), _p(), 0, _p(), 8, 16, 128, 256, _p(), _p(), NULL, NULL) == UNSUPPORTED  # bf16 only
+    assert m(_p(), _p(), _p(), _p(), 1, _p(), 8, 16, 96, 256, _p(), _p(), NULL, NULL) == UNSUPPORTED  # d % 128
+    assert m(_p(), _p(), _p(), _p(), 1, NULL, 8, 16, 128, 256, _p(), _p(), NULL, NULL) == INVALID  # counts
     c = lib.moe_unpermute_combine
     c.argtypes = [V, ctypes.c_int, V, V, V, ctypes.c_int, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, V,
                   ctypes.c_int, V]

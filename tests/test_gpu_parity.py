@@ -405,6 +405,36 @@ def test_forward_workspace_too_small_is_rejected(moe):
     assert ei.value.status == 3
 
 
+@pytest.mark.parametrize("name", ["decode_like", "block_like", "prefill_like"])
+def test_forward_replays_from_a_cuda_graph(moe, name):
+    # the whole layer is capturable (no host sync, shape-only grids, caller-owned workspace): a graph
+    # captured once replays the eager result bit for bit, and follows new data written into its input
+    T, d, E, d_ff, xd, wd, od = SMALL[name]
+    w = synth.Workload(name, T, d, E, d_ff, x_dtype=DT[xd], w_dtype=DT[wd], out_dtype=DT[od], seed=510)
+    I = {n: cuda(t) for n, t in synth.make_layer_inputs(w).items()}
+    x2 = cuda(synth.make_layer_inputs(w.scaled(seed=511))["x"])
+    args = (I["gamma"], I["W_r"], I["b"], I["W_gate"], I["W_up"], I["W_down"])
+    eager = [torch.empty((T, d), dtype=DT[od], device=DEV) for _ in range(2)]
+    ws = torch.empty(moe.forward_workspace_bytes(I["x"], I["W_r"], I["W_gate"], eager[0]), dtype=torch.uint8,
+                     device=DEV)
+    moe.moe_forward(I["x"], *args, eager[0], ws=ws)
+    moe.moe_forward(x2, *args, eager[1], ws=ws)
+    torch.cuda.synchronize()
+    x_in = I["x"].clone()
+    out = torch.empty_like(eager[0])
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        moe.moe_forward(x_in, *args, out, ws=ws)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, eager[0])
+    x_in.copy_(x2)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, eager[1])
+    del g
+
+
 def test_forward_launch_count_is_reported_and_stable(moe):
     # the library's own launch counter: one forward enqueues the same nonzero number of kernels each time
     w = synth.Workload("count", 32, 256, 16, 128)
