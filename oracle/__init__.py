@@ -17,17 +17,17 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SO = os.path.join(_HERE, "liboracle.so")
-_SRC = os.path.join(_HERE, "oracle.c")
+_SRCS = [os.path.join(_HERE, "oracle.c"), os.path.join(_HERE, "oracle_fp8.c")]
 
 F32, BF16 = 0, 1
 
 
 def build(force: bool = False) -> str:
     """Compile ``liboracle.so`` with plain gcc (no fast-math, no OpenMP)."""
-    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(_SRC):
+    if force or not os.path.exists(_SO) or any(os.path.getmtime(_SO) < os.path.getmtime(f) for f in _SRCS):
         tmp = _SO + f".tmp{os.getpid()}"
         subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-std=c11", "-fno-fast-math",
-                               "-ffp-contract=off", "-o", tmp, _SRC, "-lm"])
+                               "-ffp-contract=off", "-o", tmp, *_SRCS, "-lm"])
         os.replace(tmp, _SO)
     return _SO
 
@@ -63,6 +63,13 @@ def _L():
         L.oracle_moe_layer.argtypes = [vp, i32, i64, vp, vp, vp, vp, vp, vp, i32, i64, i64, i32, i64, dbl,
                                        vp, vp, vp, vp, vp, vp, vp]
         L.oracle_moe_layer.restype = i32
+        L.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_decode.restype = dbl
+        L.oracle_e4m3_encode.argtypes = [flt]
+        L.oracle_e4m3_encode.restype = ctypes.c_uint8
+        L.oracle_quantize_blocks.argtypes = [vp, i32, i64, i64, i64, vp, vp]
+        L.oracle_fp8_grouped_mlp.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                             vp, vp]
         _lib = L
     return _lib
 
@@ -221,3 +228,47 @@ def moe_layer(x, gamma, W_r, b, W_gate, W_up, W_down, k: int = 8, eps: float = 1
     if rc != 0:
         raise ValueError("oracle_moe_layer: bad arguments")
     return {"out": out, "idx": idx, "w": w, "z32": z32, "margin": margin}
+
+
+# --------------------------------------------------------------------------- block FP8 (oracle_fp8.c)
+def e4m3_decode(codes: torch.Tensor) -> torch.Tensor:
+    """float64 value of every E4M3 code (uint8)."""
+    c = codes.contiguous().to(torch.uint8).flatten()
+    f = _L().oracle_e4m3_decode
+    return torch.tensor([f(int(v)) for v in c.tolist()], dtype=torch.float64).reshape(codes.shape)
+
+
+def e4m3_encode(x: torch.Tensor) -> torch.Tensor:
+    """nearest E4M3 code (ties to even, saturating) of every fp32 value."""
+    v = x.contiguous().to(torch.float32).flatten()
+    f = _L().oracle_e4m3_encode
+    return torch.tensor([f(float(a)) for a in v.tolist()], dtype=torch.uint8).reshape(x.shape)
+
+
+def quantize_blocks(x: torch.Tensor, blk_rows: int):
+    """(codes uint8 [rows][cols], scales f32 [ceil(rows/blk_rows)][cols/128]) of a 2-D f32/bf16 matrix."""
+    x = _c(x)
+    rows, cols = x.shape
+    q = torch.empty((rows, cols), dtype=torch.uint8)
+    s = torch.empty(((rows + blk_rows - 1) // blk_rows, cols // 128), dtype=torch.float32)
+    _L().oracle_quantize_blocks(_p(x), _dt(x), rows, cols, blk_rows, _p(q), _p(s))
+    return q, s
+
+
+def fp8_grouped_mlp(xq, xs, counts, offsets, Wg_q, Wg_s, Wu_q, Wu_s, Wd_q, Wd_s, hq_in=None, hs_in=None):
+    """Block-FP8 grouped SwiGLU MLP: dict(h f64, hq u8, hs f32, y f64); rows outside segments are NaN / 0."""
+    xq, xs = xq.contiguous(), xs.contiguous()
+    counts, offsets = _c(counts, torch.int32), _c(offsets, torch.int32)
+    E, d_ff, d = Wg_q.shape
+    S = xq.shape[0]
+    h = torch.full((S, d_ff), float("nan"), dtype=torch.float64)
+    y = torch.full((S, d), float("nan"), dtype=torch.float64)
+    hq = torch.zeros((S, d_ff), dtype=torch.uint8)
+    hs = torch.zeros((S, d_ff // 128), dtype=torch.float32)
+    ins = [None if t is None else t.contiguous() for t in (hq_in, hs_in)]
+    _L().oracle_fp8_grouped_mlp(_p(xq), _p(xs), _p(counts), _p(offsets), E, d, d_ff,
+                                _p(Wg_q.contiguous()), _p(Wg_s.contiguous()), _p(Wu_q.contiguous()),
+                                _p(Wu_s.contiguous()), _p(Wd_q.contiguous()), _p(Wd_s.contiguous()), _p(h), _p(hq),
+                                _p(hs), _p(ins[0]), _p(ins[1]), _p(y))
+    return {"h": h, "hq": hq, "hs": hs, "y": y}
+
