@@ -45,6 +45,8 @@ def parse():
                          "for ncu captures of the same kernels, never for reported numbers")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-masked", action="store_true",
+                    help="skip the masked-layout expert MLP timing (run for workloads of <= 32 rows per expert)")
     a = ap.parse_args()
     a.warmup = max(a.warmup, 3)
     return a
@@ -313,6 +315,38 @@ def run_ours(a, w):
     roof["launch_ms"] = stage_ms["gate_up"]
     roof["peak_source"] = f"{pk['source']} (burst, kernel timed alone)"
 
+    # ---- the expert MLP on the masked layout ([E][cap][d] buffers + counts), same routing
+    masked = None
+    if not a.no_masked and w.w_dtype == torch.bfloat16 and S // E <= 32:
+        cn, of = counts.cpu(), offsets.cpu()
+        cap = int((int(cn.max()) + 15) // 16 * 16)
+        xm = torch.zeros((E, cap, w.d), dtype=w.w_dtype, device=dev)
+        for e in range(E):  # input preparation, outside the timed region
+            xm[e, :int(cn[e])] = xp[int(of[e]):int(of[e]) + int(cn[e])]
+        hm = torch.empty((E, cap, w.d_ff), dtype=w.w_dtype, device=dev)
+        ym = torch.empty((E, cap, w.d), dtype=w.w_dtype, device=dev)
+
+        def mstep():
+            moe.moe_grouped_swiglu_masked(xm, D["W_gate"], D["W_up"], D["W_down"], counts, hm, ym, dev_status=status)
+
+        for _ in range(a.warmup):
+            mstep()
+        barrier()
+        m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        m0.record()
+        for _ in range(a.steps):
+            mstep()
+        m1.record()
+        torch.cuda.synchronize()
+        if status.item() != 0:
+            raise RuntimeError(f"device status {status.item()} in the masked-layout timing")
+        mms = m0.elapsed_time(m1) / a.steps
+        mbytes = active * 3 * w.d_ff * w.d * esz + S * (2 * w.d + 2 * w.d_ff) * esz
+        masked = {"expert_mlp_ms": mms, "tokens_per_s": T / (mms / 1000.0), "cap": cap,
+                  "hbm_achieved_gbs": mbytes / (mms / 1000.0) / 1e9,
+                  "hbm_frac": mbytes / (mms / 1000.0) / 1e9 / pk["hbm_gbs"], "algorithmic_bytes": mbytes,
+                  "contiguous_expert_mlp_ms": stage_ms["gate_up"] + stage_ms["down"]}
+
     # ---- end to end through the public API with host buffers
     e2e = None
     if not a.no_e2e:
@@ -349,7 +383,7 @@ def run_ours(a, w):
                 "vs_baseline": None, "dtype": "bf16" if w.w_dtype == torch.bfloat16 else "f32",
                 "data": "synthetic", "config": config_of(w, world), "roofline": roof, "cpu_baseline": cpu,
                 "e2e": e2e, "gpu_launches": launches, "clocks": clk.summary(),
-                "stages_ms": stage_ms, "active_experts": active}
+                "stages_ms": stage_ms, "active_experts": active, "masked_layout": masked}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -82,6 +82,22 @@ typedef struct {
     const void* W_down;  /* [E][d][d_ff], w_dtype */
 } moe_weights_t;
 
+/* Block-FP8 expert weights (E4M3 codes + fp32 scales, see moe_quantize_fp8):
+ * W_*_q [E][n][k] codes, W_*_s [E][n / 128][k / 128] scales, for W_gate and
+ * W_up (n = d_ff, k = d) and W_down (n = d, k = d_ff).  gamma, W_r and b as in
+ * moe_weights_t. */
+typedef struct {
+    const float* gamma;
+    const float* W_r;
+    const float* b;
+    const uint8_t* W_gate_q;
+    const float* W_gate_s;
+    const uint8_t* W_up_q;
+    const float* W_up_s;
+    const uint8_t* W_down_q;
+    const float* W_down_s;
+} moe_weights_fp8_t;
+
 /*
  * Step 1 — RMSNorm [P1 §Norm&Residual, RMSNorm equation]:
  *   v[t][j] = gamma[j] * x[t][j] / sqrt((1/d) * sum_k x[t][k]^2 + eps)
@@ -233,6 +249,48 @@ moe_status_t moe_forward(const moe_shape_t* shape, const moe_weights_t* weights,
 
 /* Static text for a status code. */
 const char* moe_status_string(moe_status_t status);
+
+/*
+ * Block-FP8 quantisation [P5 §专家计算实现: FP8 expert GEMMs (fp8_gemm_nt) and
+ * the blockfp8 quantised experts; the page names the scheme without defining
+ * it, and this follows the usual block-FP8 layout]:
+ * x [rows][cols] (MOE_F32 or MOE_BF16, device) -> q [rows][cols] E4M3 codes and
+ * s [ceil(rows / blk_rows)][cols / 128] fp32 scales, one per block of
+ * blk_rows x 128 elements (blk_rows = 128 for weights, 1 for GEMM inputs).
+ * For a block with largest magnitude a: s = a / 448 (1 if a == 0), and each
+ * code is E4M3(x / s) rounded to nearest even, saturating at +-448 (E4M3: bias
+ * 7, no infinities, S.1111.111 is NaN).  cols % 128 == 0; x, q 16-byte aligned.
+ * A weight tensor [E][n][k] is quantised as rows = E * n (n % 128 == 0).
+ */
+moe_status_t moe_quantize_fp8(const void* x, moe_dtype_t dt, int64_t rows, int64_t cols, int32_t blk_rows, uint8_t* q,
+                              float* s, moe_stream_t stream);
+
+/*
+ * Step 4 with block-FP8 experts: for every row r of expert e's segment
+ *   g, u = dequant(xq[r]) . dequant(W_gate[e]), dequant(W_up[e])   (per feature)
+ *   h    = SiLU(g) * u, quantised per (row, 128 features) -> hq [S][d_ff], hs [S][d_ff / 128]
+ *   y[r] = dequant(hq[r]) . dequant(W_down[e])                      -> y [S][d] bf16
+ * with dequant(code) = value(code) * scale of its block, fp32 accumulation per
+ * 128-wide K block in tensor memory and fp32 promotion across blocks.  xq
+ * [S][d] codes, xs [S][d / 128] scales (moe_quantize_fp8 with blk_rows 1);
+ * w->gamma, W_r and b are not used.  d % 128 == 0, d_ff % 128 == 0.
+ */
+moe_status_t moe_grouped_swiglu_fp8(const uint8_t* xq, const float* xs, const moe_weights_fp8_t* w,
+                                    const int32_t* counts, const int32_t* offsets, int32_t S, int32_t E, int32_t d,
+                                    int32_t d_ff, uint8_t* hq, float* hs, void* y, int32_t* dev_status,
+                                    moe_stream_t stream);
+
+/*
+ * The whole layer with block-FP8 experts: as moe_forward, except that the
+ * expert path reads the normalised rows quantised per (row, 128 columns) from
+ * their fp32 values, and the expert MLP is moe_grouped_swiglu_fp8 (rows read
+ * in place through the permutation, no permuted copy).  The router is the
+ * fp32 path of moe_forward.  shape->w_dtype is ignored (expert codes are
+ * E4M3, y is bf16); x_dtype and out_dtype as in moe_forward.
+ */
+moe_status_t moe_forward_fp8(const moe_shape_t* shape, const moe_weights_fp8_t* w, const void* x, void* out,
+                             int32_t* topk_idx, float* topk_w, float* logits, void* ws, size_t* ws_bytes,
+                             int32_t* dev_status, moe_stream_t stream);
 
 /* Number of kernels the library has enqueued in this process since it was
  * loaded, over all entry points, streams and threads (successful launches

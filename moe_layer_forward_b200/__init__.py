@@ -18,15 +18,16 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoe.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m moe_layer_forward_b200.build` "
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python moe_layer_forward_b200/build.py` "
                       "(or __graft_entry__.build()); there is no fallback implementation")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
 MOE_F32, MOE_BF16 = 0, 1
-MOE_DEV_BAD_EXPERT_ID, MOE_DEV_TIMEOUT = 1, 2
+MOE_DEV_BAD_EXPERT_ID, MOE_DEV_TIMEOUT, MOE_DEV_BAD_COUNT = 1, 2, 4
 
-_vp, _i32, _f32, _szp = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.POINTER(ctypes.c_size_t)
+_vp, _i32, _i64, _f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
+_szp = ctypes.POINTER(ctypes.c_size_t)
 
 
 class MoeShape(ctypes.Structure):
@@ -37,6 +38,11 @@ class MoeShape(ctypes.Structure):
 
 class MoeWeights(ctypes.Structure):
     _fields_ = [("gamma", _vp), ("W_r", _vp), ("b", _vp), ("W_gate", _vp), ("W_up", _vp), ("W_down", _vp)]
+
+
+class MoeWeightsFP8(ctypes.Structure):
+    _fields_ = [("gamma", _vp), ("W_r", _vp), ("b", _vp), ("W_gate_q", _vp), ("W_gate_s", _vp), ("W_up_q", _vp),
+                ("W_up_s", _vp), ("W_down_q", _vp), ("W_down_s", _vp)]
 
 
 _sig = {
@@ -51,6 +57,11 @@ _sig = {
     "moe_unpermute_combine": [_vp, _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _i32, _vp],
     "moe_forward": [ctypes.POINTER(MoeShape), ctypes.POINTER(MoeWeights), _vp, _vp, _vp, _vp, _vp, _vp, _szp, _vp,
                     _vp],
+    "moe_quantize_fp8": [_vp, _i32, _i64, _i64, _i32, _vp, _vp, _vp],
+    "moe_grouped_swiglu_fp8": [_vp, _vp, ctypes.POINTER(MoeWeightsFP8), _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp,
+                               _vp, _vp, _vp],
+    "moe_forward_fp8": [ctypes.POINTER(MoeShape), ctypes.POINTER(MoeWeightsFP8), _vp, _vp, _vp, _vp, _vp, _vp, _szp,
+                        _vp, _vp],
 }
 for _name, _args in _sig.items():
     _fn = getattr(_lib, _name)
@@ -226,3 +237,65 @@ def moe_forward(x, gamma, W_r, b, W_gate, W_up, W_down, out, top_k: int = 8, eps
     _check("moe_forward", _lib.moe_forward(ctypes.byref(shp), ctypes.byref(wts), _p(x), _p(out), _p(topk_idx),
                                            _p(topk_w), _p(logits), _p(ws), ctypes.byref(n), _p(dev_status),
                                            _stream(x.device)))
+
+
+# --------------------------------------------------------------------------- block FP8 experts
+def quantize_fp8(x, blk_rows: int, q, s) -> None:
+    """E4M3 codes q and fp32 scales s of x ([..., cols]) per blk_rows x 128 block (128: weights, 1: inputs)."""
+    cols = x.shape[-1]
+    rows = x.numel() // cols
+    _check("moe_quantize_fp8", _lib.moe_quantize_fp8(_p(x), _dt(x), rows, cols, blk_rows, _p(q), _p(s),
+                                                     _stream(x.device)))
+
+
+def quantize_fp8_weights(W):
+    """(codes uint8 [E][n][k], scales f32 [E][n/128][k/128]) of an expert weight tensor, on its device."""
+    E, n, k = W.shape
+    q = torch.empty((E, n, k), dtype=torch.uint8, device=W.device)
+    s = torch.empty((E, n // 128, k // 128), dtype=torch.float32, device=W.device)
+    quantize_fp8(W, 128, q, s)
+    return q, s
+
+
+def _fp8_weights(gamma, W_r, b, Wg, Wu, Wd) -> MoeWeightsFP8:
+    return MoeWeightsFP8(_p(gamma), _p(W_r), _p(b), _p(Wg[0]), _p(Wg[1]), _p(Wu[0]), _p(Wu[1]), _p(Wd[0]),
+                         _p(Wd[1]))
+
+
+def moe_grouped_swiglu_fp8(xq, xs, Wg, Wu, Wd, counts, offsets, hq, hs, y, dev_status=None) -> None:
+    """Block-FP8 expert MLP; Wg/Wu/Wd are (codes, scales) pairs, xq/xs the input rows' codes and scales."""
+    S, d = xq.shape
+    E, d_ff, _ = Wg[0].shape
+    w = _fp8_weights(None, None, None, Wg, Wu, Wd)
+    _check("moe_grouped_swiglu_fp8",
+           _lib.moe_grouped_swiglu_fp8(_p(xq), _p(xs), ctypes.byref(w), _p(counts), _p(offsets), S, E, d, d_ff,
+                                       _p(hq), _p(hs), _p(y), _p(dev_status), _stream(xq.device)))
+
+
+def _shape_fp8(x, Wg_q, out, top_k, eps, E) -> MoeShape:
+    T, d = x.shape
+    return MoeShape(T, d, E, top_k, Wg_q.shape[1], eps, _dt(x), MOE_BF16, _dt(out))
+
+
+def forward_fp8_workspace_bytes(x, W_r, Wg_q, out, top_k: int = 8, eps: float = 1e-5) -> int:
+    shp = _shape_fp8(x, Wg_q, out, top_k, eps, W_r.shape[0])
+    w = MoeWeightsFP8()
+    n = ctypes.c_size_t(0)
+    _check("moe_forward_fp8", _lib.moe_forward_fp8(ctypes.byref(shp), ctypes.byref(w), None, None, None, None, None,
+                                                   None, ctypes.byref(n), None, _stream(x.device)))
+    return int(n.value)
+
+
+def moe_forward_fp8(x, gamma, W_r, b, Wg, Wu, Wd, out, top_k: int = 8, eps: float = 1e-5, topk_idx=None,
+                    topk_w=None, logits=None, ws=None, dev_status=None) -> None:
+    """out = x + MoE(RMSNorm(x)) with block-FP8 experts (Wg/Wu/Wd: (codes, scales) pairs)."""
+    shp = _shape_fp8(x, Wg[0], out, top_k, eps, W_r.shape[0])
+    w = _fp8_weights(gamma, W_r, b, Wg, Wu, Wd)
+    if ws is None:
+        ws = torch.empty(max(forward_fp8_workspace_bytes(x, W_r, Wg[0], out, top_k, eps), 1), dtype=torch.uint8,
+                         device=x.device)
+    n = ctypes.c_size_t(ws.numel())
+    _check("moe_forward_fp8", _lib.moe_forward_fp8(ctypes.byref(shp), ctypes.byref(w), _p(x), _p(out), _p(topk_idx),
+                                                   _p(topk_w), _p(logits), _p(ws), ctypes.byref(n), _p(dev_status),
+                                                   _stream(x.device)))
+

@@ -358,4 +358,123 @@ moe_status_t moe_forward(const moe_shape_t* shape, const moe_weights_t* wts, con
     return cuda_status(launch_combine(c, y, wdt, token_slot, wgt, x, xdt, T, d, k, out, shape->out_dtype));
 }
 
+
+// ----------------------------------------------------------------------------- block FP8
+moe_status_t moe_quantize_fp8(const void* x, moe_dtype_t dt, int64_t rows, int64_t cols, int32_t blk_rows, uint8_t* q,
+                              float* s, moe_stream_t stream) {
+    if (!valid_dt(dt) || rows < 0 || cols <= 0 || (blk_rows != 1 && blk_rows != 128)) return MOE_ERR_INVALID_ARG;
+    if (cols % 128 != 0 || rows * cols >= (int64_t(1) << 40)) return MOE_ERR_UNSUPPORTED;
+    if (rows == 0) return MOE_OK;
+    if (!x || !q || !s || !aligned16(x) || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+    Ctx c;
+    moe_status_t st = make_ctx(stream, c);
+    if (st != MOE_OK) return st;
+    return cuda_status(launch_quant_fp8(c, x, dt, rows, cols, blk_rows, q, s));
+}
+
+namespace {
+moe_status_t check_fp8_weights(const moe_weights_fp8_t* w) {
+    if (!w || !w->W_gate_q || !w->W_gate_s || !w->W_up_q || !w->W_up_s || !w->W_down_q || !w->W_down_s)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(w->W_gate_q) || !aligned16(w->W_up_q) || !aligned16(w->W_down_q)) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+}  // namespace
+
+moe_status_t moe_grouped_swiglu_fp8(const uint8_t* xq, const float* xs, const moe_weights_fp8_t* w,
+                                    const int32_t* counts, const int32_t* offsets, int32_t S, int32_t E, int32_t d,
+                                    int32_t d_ff, uint8_t* hq, float* hs, void* y, int32_t* dev_status,
+                                    moe_stream_t stream) {
+    moe_status_t st = check_expert_shape(MOE_BF16, S, E, d, d_ff);
+    if (st != MOE_OK) return st;
+    if (S == 0) return MOE_OK;
+    st = check_fp8_weights(w);
+    if (st != MOE_OK) return st;
+    if (!xq || !xs || !counts || !offsets || !hq || !hs || !y || !aligned16(xq) || !aligned16(hq) || !aligned16(y))
+        return MOE_ERR_INVALID_ARG;
+    Ctx c;
+    st = make_ctx(stream, c);
+    if (st != MOE_OK) return st;
+    st = cuda_status(launch_gate_up_fp8(c, xq, xs, nullptr, w->W_gate_q, w->W_gate_s, w->W_up_q, w->W_up_s, counts,
+                                        offsets, S, E, d, d_ff, hq, hs, dev_status));
+    if (st != MOE_OK) return st;
+    return cuda_status(
+        launch_down_fp8(c, hq, hs, w->W_down_q, w->W_down_s, counts, offsets, S, E, d, d_ff, y, dev_status));
+}
+
+moe_status_t moe_forward_fp8(const moe_shape_t* shape, const moe_weights_fp8_t* w, const void* x, void* out,
+                             int32_t* topk_idx, float* topk_w, float* logits, void* ws, size_t* ws_bytes,
+                             int32_t* dev_status, moe_stream_t stream) {
+    if (!shape || !w || !ws_bytes) return MOE_ERR_INVALID_ARG;
+    const int T = shape->T, d = shape->d, E = shape->E, k = shape->top_k, d_ff = shape->d_ff;
+    if (!valid_dt(shape->x_dtype) || !valid_dt(shape->out_dtype)) return MOE_ERR_INVALID_ARG;
+    moe_status_t st = check_router_shape(T, d, E, k);
+    if (st != MOE_OK) return st;
+    if ((int64_t)T * k > INT32_MAX / 2) return MOE_ERR_UNSUPPORTED;
+    const int S = T * k;
+    st = check_expert_shape(MOE_BF16, S, E, d, d_ff);
+    if (st != MOE_OK) return st;
+    Ctx c;
+    st = make_ctx(stream, c);
+    if (st != MOE_OK) return st;
+    const RouterPlan plan = plan_router(T, d, E, c.num_sms);
+
+    Carve cv(ws);
+    uint8_t* vq = static_cast<uint8_t*>(cv.take((size_t)T * d));
+    float* vs = static_cast<float*>(cv.take((size_t)T * (d / 128) * sizeof(float)));
+    float* rstd = static_cast<float*>(cv.take((size_t)T * sizeof(float)));
+    float* partial = static_cast<float*>(cv.take(plan.partial_bytes));
+    float* wsplit = static_cast<float*>(cv.take(plan.wsplit_bytes));
+    int32_t* idx_ws = static_cast<int32_t*>(cv.take((size_t)S * sizeof(int32_t)));
+    float* wgt_ws = static_cast<float*>(cv.take((size_t)S * sizeof(float)));
+    int32_t* idx = topk_idx ? topk_idx : idx_ws;
+    float* wgt = topk_w ? topk_w : wgt_ws;
+    int32_t* hist = static_cast<int32_t*>(cv.take(permute_ws_bytes(T, E)));
+    int32_t* counts = static_cast<int32_t*>(cv.take((size_t)E * sizeof(int32_t)));
+    int32_t* offsets = static_cast<int32_t*>(cv.take((size_t)(E + 1) * sizeof(int32_t)));
+    int32_t* slot_token = static_cast<int32_t*>(cv.take((size_t)S * sizeof(int32_t)));
+    int32_t* token_slot = static_cast<int32_t*>(cv.take((size_t)S * sizeof(int32_t)));
+    uint8_t* hq = static_cast<uint8_t*>(cv.take((size_t)S * d_ff));
+    float* hs = static_cast<float*>(cv.take((size_t)S * (d_ff / 128) * sizeof(float)));
+    void* y = cv.take((size_t)S * d * 2);
+    bool query = false;
+    st = check_ws(ws, ws_bytes, cv.off, &query);
+    if (st != MOE_OK || query) return st;
+
+    if (T > 0) {
+        if (!x || !out || !w->gamma || !w->W_r || !w->b) return MOE_ERR_INVALID_ARG;
+        if (!aligned16(x) || !aligned16(out) || !aligned16(w->gamma) || !aligned16(w->W_r)) return MOE_ERR_INVALID_ARG;
+        st = check_fp8_weights(w);
+        if (st != MOE_OK) return st;
+    }
+    if (dev_status) {
+        st = cuda_status(cudaMemsetAsync(dev_status, 0, sizeof(int32_t), c.stream));
+        if (st != MOE_OK) return st;
+    }
+    if (T == 0) return MOE_OK;
+    const int xdt = shape->x_dtype;
+    // 1. RMSNorm: codes of the normalised rows for the experts, 1/rms for the router
+    st = cuda_status(launch_rmsnorm_quant(c, x, xdt, w->gamma, T, d, shape->eps, vq, vs, rstd));
+    if (st != MOE_OK) return st;
+    // 2. router on the unrounded fp32 normalised rows
+    st = cuda_status(
+        launch_router_logits(c, plan, x, xdt, rstd, w->gamma, w->W_r, T, d, E, partial, wsplit, dev_status));
+    if (st != MOE_OK) return st;
+    st = cuda_status(launch_router_topk(c, plan, partial, w->b, T, E, k, idx, wgt, logits, nullptr));
+    if (st != MOE_OK) return st;
+    // 3. permutation maps only: the gate/up GEMM reads the code rows in place
+    st = cuda_status(launch_permute(c, nullptr, MOE_BF16, idx, T, d, E, k, counts, offsets, slot_token, token_slot,
+                                    nullptr, hist, dev_status));
+    if (st != MOE_OK) return st;
+    // 4. block-FP8 SwiGLU MLP
+    st = cuda_status(launch_gate_up_fp8(c, vq, vs, slot_token, w->W_gate_q, w->W_gate_s, w->W_up_q, w->W_up_s, counts,
+                                        offsets, S, E, d, d_ff, hq, hs, dev_status));
+    if (st != MOE_OK) return st;
+    st = cuda_status(
+        launch_down_fp8(c, hq, hs, w->W_down_q, w->W_down_s, counts, offsets, S, E, d, d_ff, y, dev_status));
+    if (st != MOE_OK) return st;
+    // 5. weighted un-permute + residual
+    return cuda_status(launch_combine(c, y, MOE_BF16, token_slot, wgt, x, xdt, T, d, k, out, shape->out_dtype));
+}
+
 }  // extern "C"

@@ -89,6 +89,19 @@ cudaError_t launch_gate_up_bf16_pair(const Ctx& c, const void* xp, const void* W
                                      void* h, int32_t* status);
 cudaError_t launch_down_bf16_pair(const Ctx& c, const void* h, const void* Wd, const int32_t* counts,
                                   const int32_t* offsets, int S, int E, int d, int d_ff, void* y, int32_t* status);
+// Block-FP8 experts (expert_fp8.cu): E4M3 codes, fp32 scales per 128 x 128 weight block and per
+// (row, 128 columns) of a GEMM input
+cudaError_t launch_quant_fp8(const Ctx& c, const void* x, int dt, int64_t rows, int64_t cols, int blk_rows,
+                             uint8_t* q, float* s);
+cudaError_t launch_rmsnorm_quant(const Ctx& c, const void* x, int x_dt, const float* gamma, int T, int d, float eps,
+                                 uint8_t* q, float* s, float* rstd);
+cudaError_t launch_gate_up_fp8(const Ctx& c, const uint8_t* xq, const float* xs, const int32_t* gather,
+                               const uint8_t* Wg, const float* Wg_s, const uint8_t* Wu, const float* Wu_s,
+                               const int32_t* counts, const int32_t* offsets, int S, int E, int d, int d_ff,
+                               uint8_t* hq, float* hs, int32_t* status);
+cudaError_t launch_down_fp8(const Ctx& c, const uint8_t* hq, const float* hs, const uint8_t* Wd, const float* Wd_s,
+                            const int32_t* counts, const int32_t* offsets, int S, int E, int d, int d_ff, void* y,
+                            int32_t* status);
 cudaError_t launch_gate_up_f32(const Ctx& c, const float* xp, const float* Wg, const float* Wu, const int32_t* counts,
                                const int32_t* offsets, int S, int E, int d, int d_ff, float* h);
 cudaError_t launch_down_f32(const Ctx& c, const float* h, const float* Wd, const int32_t* counts,

@@ -145,6 +145,12 @@ def test_expert_and_combine_reject_bad_shapes_on_host(lib):
     assert m(_p(), _p(), _p(), _p(), 0, _p(), 8, 16, 128, 256, _p(), _p(), NULL, NULL) == UNSUPPORTED  # bf16 only
     assert m(_p(), _p(), _p(), _p(), 1, _p(), 8, 16, 96, 256, _p(), _p(), NULL, NULL) == UNSUPPORTED  # d % 128
     assert m(_p(), _p(), _p(), _p(), 1, NULL, 8, 16, 128, 256, _p(), _p(), NULL, NULL) == INVALID  # counts
+    qz = lib.moe_quantize_fp8
+    qz.argtypes = [V, ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, V, V, V]
+    assert qz(_p(), 1, 64, 256, 64, _p(), _p(), NULL) == INVALID  # block of 1 or 128 rows
+    assert qz(_p(), 1, 64, 200, 128, _p(), _p(), NULL) == UNSUPPORTED  # cols % 128
+    assert qz(_p(), 7, 64, 256, 1, _p(), _p(), NULL) == INVALID  # dtype
+    assert qz(_p(), 1, 0, 256, 1, _p(), _p(), NULL) == OK  # nothing to do
     c = lib.moe_unpermute_combine
     c.argtypes = [V, ctypes.c_int, V, V, V, ctypes.c_int, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, V,
                   ctypes.c_int, V]
