@@ -18,10 +18,10 @@
 //       the expert's rows (tokens) are N <= R.  K runs in 128-wide blocks: a stage
 //       holds one 128-byte swizzled row slice per operand (exactly one scale block),
 //       and the MMA thread issues 4 kind::f8f6f4 MMAs (K = 32) per operand into one
-//       of two tensor-memory chunk buffers.  Four epilogue warps promote each chunk
+//       of eight tensor-memory chunk buffers.  Four epilogue warps promote each chunk
 //       into fp32 register sums with s_w * s_a(row) and release the buffer, so the
-//       next block's MMAs overlap the promotion.  Gate/up ends with SiLU(g) * u and
-//       quantises h per (row, 128 features) for the down projection (an amax over
+//       next blocks' MMAs overlap the promotion (whose scale loads run one block
+//       ahead).  Gate/up ends with SiLU(g) * u and quantises h per (row, 128 features) for the down projection (an amax over
 //       the 128 weight rows of the tile: warp shuffles, then the 4 warps in shared
 //       memory); down ends with bf16 y.  Activation rows are copied by four loader
 //       warps (16-byte cp.async into the swizzled layout, optionally through the
@@ -188,7 +188,9 @@ struct Cfg {
     static constexpr int STAGES = STAGES_MAX > 8 ? 8 : STAGES_MAX;
     static_assert(STAGES >= 3, "pipeline depth");
     static constexpr int CB = NUM_A * R;  // columns of one chunk buffer: gate | up
-    static constexpr int TMEM_COLS = 2 * CB <= 32 ? 32 : (2 * CB <= 64 ? 64 : 128);
+    static constexpr int NBUF = 8;        // chunk buffers: the MMAs run up to 7 K blocks ahead of the promotion
+    static constexpr int TMEM_COLS = NBUF * CB <= 128 ? 128 : (NBUF * CB <= 256 ? 256 : 512);
+    static_assert(NBUF * CB <= 512, "tensor memory");
     static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + AUX_BYTES;
 };
 
@@ -212,8 +214,8 @@ struct Args {
 struct Aux {
     uint64_t full[8];
     uint64_t empty[8];
-    uint64_t cfull[2];
-    uint64_t cempty[2];
+    uint64_t cfull[8];
+    uint64_t cempty[8];
     uint64_t drain;
     uint64_t redbar;  // the 4 epilogue warps' per-tile rendezvous on red
     uint32_t tmem_slot;
@@ -255,7 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(smem_u32(&aux.full[s]), 2);  // weight TMA (with its bytes) + the activation loader
             mbar_init(smem_u32(&aux.empty[s]), 1);
         }
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < C::NBUF; ++c) {
             mbar_init(smem_u32(&aux.cfull[c]), 1);
             mbar_init(smem_u32(&aux.cempty[c]), 4);
         }
@@ -358,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int rows = min(R, aux.cnt[e] - rb * R);
             const uint32_t idesc = idesc_e4m3(128, (rows + 15) & ~15);
             for (int kb = 0; kb < nk; ++kb, ++q) {
-                const uint32_t c = q & 1u, use = q >> 1;
+                const uint32_t c = q % C::NBUF, use = q / C::NBUF;
                 if (!warp_wait(smem_u32(&aux.full[stage]), phase, abort_flag) ||
                     !warp_wait(smem_u32(&aux.cempty[c]), (use & 1u) ^ 1u, abort_flag)) {
                     give_up();
@@ -451,8 +453,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             float g[R], u[R];
 #pragma unroll
             for (int n = 0; n < R; ++n) g[n] = u[n] = 0.f;
+            // scales of the next block load while this block's chunk is awaited
+            float sw1_n = __ldg(s1), sw2_n = SWIGLU ? __ldg(s2) : 0.f;
+            float sa_n = lane < rows ? __ldg(p.act_s + (int64_t)my_row * nk) : 0.f;
             for (int kb = 0; kb < nk; ++kb, ++q) {
-                const uint32_t c = q & 1u, use = q >> 1;
+                const float sw1 = sw1_n, sw2 = sw2_n, my_sa = sa_n;
+                if (kb + 1 < nk) {
+                    sw1_n = __ldg(s1 + kb + 1);
+                    if (SWIGLU) sw2_n = __ldg(s2 + kb + 1);
+                    sa_n = lane < rows ? __ldg(p.act_s + (int64_t)my_row * nk + kb + 1) : 0.f;
+                }
+                const uint32_t c = q % C::NBUF, use = q / C::NBUF;
                 if (!warp_wait(smem_u32(&aux.cfull[c]), use & 1u, abort_flag)) {
                     give_up();
                     ok = false;
@@ -468,9 +479,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&aux.cempty[c]));
-                const float sw1 = __ldg(s1 + kb);
-                const float sw2 = SWIGLU ? __ldg(s2 + kb) : 0.f;
-                const float my_sa = lane < rows ? __ldg(p.act_s + (int64_t)my_row * nk + kb) : 0.f;
 #pragma unroll
                 for (int n = 0; n < R; ++n) {
                     const float sa = __shfl_sync(0xffffffffu, my_sa, n);
