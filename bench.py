@@ -19,6 +19,7 @@ import datetime
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -45,6 +46,8 @@ def parse():
                          "for ncu captures of the same kernels, never for reported numbers")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-fp8", action="store_true",
+                    help="skip the block-FP8 layer timing (run for bf16 workloads of <= 32 rows per expert)")
     ap.add_argument("--no-masked", action="store_true",
                     help="skip the masked-layout expert MLP timing (run for workloads of <= 32 rows per expert)")
     a = ap.parse_args()
@@ -132,12 +135,20 @@ class Clocks:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def kernel_code_sha() -> str:
+    """Hash of the dominant kernel's source code with comments and whitespace removed."""
+    text = "".join(open(f, encoding="utf-8").read() for f in GEMM_SRC)
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return hashlib.sha256(" ".join(text.split()).encode()).hexdigest()[:16]
+
+
 def traffic_for(workload: str):
-    """DRAM bytes per launch of the dominant kernel from the committed ncu summary, if the kernel is unchanged."""
+    """DRAM bytes per launch of the dominant kernel from the committed ncu summary, if its code is unchanged."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
     j = json.load(open(TRAFFIC_FILE))
-    sha = hashlib.sha256(b"".join(open(f, "rb").read() for f in GEMM_SRC)).hexdigest()[:16]
+    sha = kernel_code_sha()
     e = j.get(workload)
     if not e or e.get("source_sha") != sha:
         return None
@@ -347,6 +358,39 @@ def run_ours(a, w):
                   "hbm_frac": mbytes / (mms / 1000.0) / 1e9 / pk["hbm_gbs"], "algorithmic_bytes": mbytes,
                   "contiguous_expert_mlp_ms": stage_ms["gate_up"] + stage_ms["down"]}
 
+    # ---- the layer with block-FP8 experts (weights quantised on the device beforehand)
+    fp8 = None
+    if not a.no_fp8 and w.w_dtype == torch.bfloat16 and S // E <= 32:
+        Wq = [moe.quantize_fp8_weights(D[n]) for n in ("W_gate", "W_up", "W_down")]
+        out8 = torch.empty_like(out)
+        ws8 = torch.empty(moe.forward_fp8_workspace_bytes(D["x"], D["W_r"], Wq[0][0], out8, k, w.eps),
+                          dtype=torch.uint8, device=dev)
+
+        def fstep():
+            moe.moe_forward_fp8(D["x"], D["gamma"], D["W_r"], D["b"], *Wq, out8, top_k=k, eps=w.eps, ws=ws8,
+                                dev_status=status)
+
+        for _ in range(a.warmup):
+            fstep()
+        barrier()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record()
+        for _ in range(a.steps):
+            fstep()
+        g1.record()
+        torch.cuda.synchronize()
+        if status.item() != 0:
+            raise RuntimeError(f"device status {status.item()} in the FP8 timing")
+        fms = g0.elapsed_time(g1) / a.steps
+        # algorithmic bytes: active experts' codes and scales, the input, the output and the router weights
+        fbytes = active * 3 * w.d_ff * w.d * (1 + 4 / (128 * 128)) + T * w.d * (D["x"].element_size() +
+                                                                                 out.element_size()) + E * w.d * 4
+        fp8 = {"ms_per_step": fms, "tokens_per_s": T / (fms / 1000.0), "dtype": "e4m3 experts, fp32 router",
+               "algorithmic_bytes": fbytes, "hbm_achieved_gbs": fbytes / (fms / 1000.0) / 1e9,
+               "hbm_frac": fbytes / (fms / 1000.0) / 1e9 / pk["hbm_gbs"],
+               "vs_bf16_layer": ms_per_step / fms}
+        del Wq
+
     # ---- end to end through the public API with host buffers
     e2e = None
     if not a.no_e2e:
@@ -383,7 +427,7 @@ def run_ours(a, w):
                 "vs_baseline": None, "dtype": "bf16" if w.w_dtype == torch.bfloat16 else "f32",
                 "data": "synthetic", "config": config_of(w, world), "roofline": roof, "cpu_baseline": cpu,
                 "e2e": e2e, "gpu_launches": launches, "clocks": clk.summary(),
-                "stages_ms": stage_ms, "active_experts": active, "masked_layout": masked}
+                "stages_ms": stage_ms, "active_experts": active, "masked_layout": masked, "fp8_layer": fp8}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -33,7 +33,7 @@
 //     rows-as-M; for down, whose weight tile is one 128-row operand, it
 //     leaves the tensor pipe co-limiting and rows-as-M is ~30% faster.
 //
-// Warp roles (192 threads, 1 CTA per SM):
+// Warp roles (1 CTA per SM; 192 threads, 320 for weights-as-M):
 //   warp 0      TMA producer: a STAGES-deep ring of 64-wide K slices (128-byte
 //               swizzled rows), one mbarrier pair (full/empty) per stage.
 //   warp 1      owns the tensor-memory allocation; lane 0 issues tcgen05.mma
@@ -42,6 +42,9 @@
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator (each warp its 32 TMEM
 //               lanes), SiLU(g)*u in fp32, bf16 stores.  Two accumulator
 //               buffers let the epilogue of one tile overlap the next tile's MMAs.
+//   warps 6..9  (weights-as-M with Args::gather) copy each stage's token rows
+//               straight from V through the slot -> token map (cp.async).
+// Masked layout (Args::cap > 0): expert e's rows start at e * cap.
 // Every wait is bounded (globaltimer); a wait that gives up raises
 // DEV_TIMEOUT in the status word and all roles unwind, drain in-flight copies
 // and MMAs, free tensor memory and exit.
