@@ -1,0 +1,47 @@
+"""Tensor-parallel experts: every expert's MLP split along d_ff across ranks.
+
+"推理计算流梳理", §实际 MLP 计算策略: with tensor parallelism the gate and up
+projections are split by columns (each rank holds a slice of the d_ff
+features) and the down projection by rows (the matching slice of its input),
+so each rank produces a partial sum of the output that one reduction
+completes.  Applied here to every expert of the MoE layer.
+
+Rank r of N holds W_gate[:, r*F:(r+1)*F, :], W_up[:, r*F:(r+1)*F, :] and
+W_down[:, :, r*F:(r+1)*F] with F = d_ff / N (a multiple of 128).  Every rank
+holds all tokens.  One step:
+
+  1. RMSNorm, router top-k and the permutation, identical on every rank;
+  2. the grouped SwiGLU MLP on the rank's d_ff slice: a partial y;
+  3. the weighted combine of the partial y in fp32, with the residual added on
+     rank 0 only, then one fp32 all-reduce (sum) across the ranks, and a cast
+     to the output dtype.
+
+All arithmetic runs in the library's kernels (``ops``, as in ``ep``); the
+reduction is ``torch.distributed.all_reduce`` (NCCL on GPUs).
+"""
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+from .ep import CudaOps
+
+
+def tp_forward(x, gamma, W_r, b, W_gate_slice, W_up_slice, W_down_slice, top_k: int = 8, eps: float = 1e-5,
+               group=None, ops=None, out_dtype=None):
+    """out = x + MoE(RMSNorm(x)) with this rank's d_ff slice of every expert (collective over ``group``)."""
+    ops = ops or CudaOps()
+    rank = dist.get_rank(group)
+    E = W_gate_slice.shape[0]
+    out_dtype = out_dtype or x.dtype
+    if W_down_slice.shape[2] != W_gate_slice.shape[1]:
+        raise ValueError("W_down's slice must match the gate/up feature slice")
+    v32 = ops.rmsnorm(x, gamma, eps, torch.float32)
+    vx = ops.rmsnorm(x, gamma, eps, W_gate_slice.dtype)
+    idx, w = ops.router(v32, W_r, b, top_k)
+    counts, offsets, token_slot, xp = ops.permute(vx, idx, E)
+    y_part = ops.grouped_swiglu(xp, W_gate_slice, W_up_slice, W_down_slice, counts, offsets)
+    residual = x if rank == 0 else torch.zeros_like(x)
+    part = ops.combine(y_part, token_slot, w, residual, torch.float32)
+    dist.all_reduce(part, op=dist.ReduceOp.SUM, group=group)
+    return part.to(out_dtype)

@@ -1,10 +1,14 @@
-"""Expert-parallel orchestration (moe_layer_forward_b200.ep) on CPU ranks.
+"""Expert- and tensor-parallel orchestration (moe_layer_forward_b200.ep, .tp)
+on CPU ranks.
 
-The exchange logic (count and row All-to-Alls, the local re-permutation, the
-way back) runs on 2 and 4 gloo ranks, each with its share of the tokens and of
-the experts.  The steps are the fp64 oracle's (ops on CPU tensors): every row
-is computed by the same arithmetic with or without expert parallelism, so the
-concatenated outputs must equal the single-process layer exactly.
+Expert parallel: the exchange logic (count and row All-to-Alls, the local
+re-permutation, the way back) runs on 2 and 4 gloo ranks, each with its share
+of the tokens and of the experts.  The steps are the fp64 oracle's (ops on CPU
+tensors): every row is computed by the same arithmetic with or without expert
+parallelism, so the concatenated outputs must equal the single-process layer
+exactly.  Tensor parallel: each rank holds a d_ff slice of every expert; the
+all-reduced result must equal the single-process layer up to the regrouping
+of the down projection's sum.
 """
 import os
 import socket
@@ -111,3 +115,54 @@ def test_expert_parallel_layer_equals_the_single_process_layer(world):
     assert torch.equal(merged, ref)
     # every routed row leaves and comes back once
     assert sum(x["sent"] for x in r) == sum(x["received"] for x in r) == w.T * w.top_k
+
+
+# --------------------------------------------------------------------------- tensor-parallel experts
+def _tp_inputs():
+    sys.path.insert(0, ROOT)
+    import synth
+
+    w = synth.Workload("tp", 20, 256, 8, 512, x_dtype=torch.float32, w_dtype=torch.float32,
+                       out_dtype=torch.float32, seed=43)
+    return w, synth.make_layer_inputs(w)
+
+
+def _tp_worker(rank, world, port, outdir):
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import datetime
+
+    import torch.distributed as dist
+
+    from moe_layer_forward_b200 import tp
+
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    w, I = _tp_inputs()
+    F = w.d_ff // world
+    f = slice(rank * F, (rank + 1) * F)
+    out = tp.tp_forward(I["x"], I["gamma"], I["W_r"], I["b"], I["W_gate"][:, f].contiguous(),
+                        I["W_up"][:, f].contiguous(), I["W_down"][:, :, f].contiguous(), top_k=w.top_k, eps=w.eps,
+                        ops=OracleOps())
+    torch.save({"out": out}, os.path.join(outdir, f"r{rank}.pt"))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_tensor_parallel_layer_equals_the_single_process_layer(world):
+    sys.path.insert(0, ROOT)
+    w, I = _tp_inputs()
+    ops = OracleOps()
+    v32 = ops.rmsnorm(I["x"], I["gamma"], w.eps, torch.float32)
+    idx, wt = ops.router(v32, I["W_r"], I["b"], w.top_k)
+    counts, offsets, token_slot, xp = ops.permute(v32, idx, w.E)
+    y = ops.grouped_swiglu(xp, I["W_gate"], I["W_up"], I["W_down"], counts, offsets)
+    ref = ops.combine(y, token_slot, wt, I["x"], torch.float64)
+    with tempfile.TemporaryDirectory() as d:
+        mp.start_processes(_tp_worker, args=(world, _free_port(), d), nprocs=world, join=True, start_method="spawn")
+        r = [torch.load(os.path.join(d, f"r{k}.pt"))["out"] for k in range(world)]
+    for k in range(world):  # every rank holds the whole result
+        assert torch.equal(r[k], r[0])
+    # the d_ff split only regroups the down projection's sum; fp32 partials add fp32 rounding
+    assert torch.allclose(r[0].double(), ref, rtol=1e-5, atol=1e-5)

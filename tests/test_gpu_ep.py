@@ -1,8 +1,9 @@
-"""Expert-parallel forward on the GPU with the library's kernels and NCCL, one
-rank (the only GPU a test here has): with every expert local the exchange is
-an identity, and the result must equal moe_forward bit for bit (same router
-arithmetic, same GEMM tiles, same combine).  Runs in a spawned process so the
-NCCL group does not outlive the test."""
+"""Expert- and tensor-parallel forwards on the GPU with the library's kernels
+and NCCL, one rank (the only GPU a test here has): with every expert and
+feature local the exchange and the reduction are identities, and the result
+must equal moe_forward bit for bit (same router arithmetic, same GEMM tiles,
+same combine).  Runs in a spawned process so the NCCL group does not outlive
+the test."""
 import os
 import socket
 import sys
@@ -43,17 +44,22 @@ def _worker(rank, port, outdir, shape):
     out = torch.empty_like(out_ep)
     moe.moe_forward(D["x"], D["gamma"], D["W_r"], D["b"], D["W_gate"], D["W_up"], D["W_down"], out, top_k=w.top_k,
                     eps=w.eps)
+    from moe_layer_forward_b200 import tp
+
+    out_tp = tp.tp_forward(D["x"], D["gamma"], D["W_r"], D["b"], D["W_gate"], D["W_up"], D["W_down"], top_k=w.top_k,
+                           eps=w.eps)
     torch.cuda.synchronize()
-    torch.save({"equal": torch.equal(out_ep, out), "rows": stats.rows_received}, os.path.join(outdir, "r.pt"))
+    torch.save({"equal": torch.equal(out_ep, out), "tp_equal": torch.equal(out_tp, out), "rows": stats.rows_received},
+               os.path.join(outdir, "r.pt"))
     dist.destroy_process_group()
 
 
 @pytest.mark.parametrize("shape", [(96, 512, 64, 256), (1200, 256, 8, 256)])  # weights-as-M; CTA pairs
-def test_single_rank_expert_parallel_equals_moe_forward(shape):
+def test_single_rank_expert_and_tensor_parallel_equal_moe_forward(shape):
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
     with tempfile.TemporaryDirectory() as d:
         mp.start_processes(_worker, args=(_free_port(), d, shape), nprocs=1, join=True, start_method="spawn")
         r = torch.load(os.path.join(d, "r.pt"))
-    assert r["equal"]
+    assert r["equal"] and r["tp_equal"]
     assert r["rows"] == shape[0] * 8
