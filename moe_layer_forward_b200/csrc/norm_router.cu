@@ -19,7 +19,8 @@
 //   router_topk_kernel   one warp per token: sums the K-split partials in split
 //                        order, scores sigmoid(z)+b in fp32 (sigmoid in double,
 //                        rounded once), then k rounds of a warp-shuffle argmax
-//                        (ties to the lower index) plus one more for the margin.
+//                        over (score, index) packed in 64 bits (ties to the lower
+//                        index) plus one more for the margin.
 //   router_topk_token_kernel  the same for few tokens: a CTA per token, a thread
 //                        per expert for the split sum, then one warp selects.
 #include <math.h>
@@ -117,30 +118,54 @@ cudaError_t launch_rmsnorm(const Ctx& c, const void* x, int x_dt, const float* g
 }
 
 // ----------------------------------------------------------------------------- top-k
-__device__ __forceinline__ bool better(float ka, int ea, float kb, int eb) { return ka > kb || (ka == kb && ea < eb); }
-
 // Scores, top-k selection and weights of token t from its logits z[j] = z(lane + 32 j), by one
 // warp: sigmoid in double rounded once to fp32, + b in fp32, k rounds of a warp-shuffle argmax
 // (ties to the lower index) and one more for the margin to the first expert left out.
+// Order-preserving 32-bit image of a non-NaN float (a larger float gives a larger unsigned; -0 is +0).
+__device__ __forceinline__ uint32_t ordered_bits(float f) {
+    const uint32_t u = __float_as_uint(f + 0.0f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float from_ordered(uint32_t o) {
+    return __uint_as_float((o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o);
+}
+__device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t v, int o) {
+    const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, o);
+    const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v >> 32), o);
+    return ((uint64_t)hi << 32) | lo;
+}
+
 __device__ __forceinline__ void select_topk_warp(const float (&z)[8], int lane, int t, const float* __restrict__ b,
                                                  int E, int k, int32_t* __restrict__ idx, float* __restrict__ w,
                                                  float* __restrict__ logits, float* __restrict__ margin) {
-    float key[8];
-    uint32_t taken = 0;  // bit j: entry lane + 32 j unavailable
+    // candidate of entry e = lane + 32 j: (ordered score << 32) | ~e, so that the largest value is the
+    // highest score and, among equal scores, the lowest expert index; 0 = no candidate
+    uint64_t cand[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         const int e = lane + 32 * j;
-        key[j] = -INFINITY;
+        cand[j] = 0;
         if (e < E) {
             const float acc = z[j];
             if (logits) logits[(int64_t)t * E + e] = acc;
             const float sg = (float)(1.0 / (1.0 + exp(-(double)acc)));
             const float sc = sg + b[e];
-            key[j] = isnan(sc) ? -INFINITY : sc;
-        } else {
-            taken |= 1u << j;
+            cand[j] = ((uint64_t)ordered_bits(isnan(sc) ? -INFINITY : sc) << 32) | (0xFFFFFFFFu - (uint32_t)e);
         }
     }
+    // this lane's best remaining candidate and its logit
+    uint64_t best = 0;
+    float best_z = 0.f;
+    auto refresh = [&]() {
+        best = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (cand[j] > best) {
+                best = cand[j];
+                best_z = z[j];
+            }
+    };
+    refresh();
     int sel_e[kMaxTopK];
     float sel_z[kMaxTopK];
     float kth = 0.f, next = INFINITY;
@@ -148,52 +173,45 @@ __device__ __forceinline__ void select_topk_warp(const float (&z)[8], int lane, 
 #pragma unroll
     for (int r = 0; r < kMaxTopK + 1; ++r) {
         if (r >= rounds) break;
-        float bk = -INFINITY;
-        int be = 0x7fffffff;
-        float bz = 0.f;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int e = lane + 32 * j;
-            if (!(taken & (1u << j)) && better(key[j], e, bk, be)) {
-                bk = key[j];
-                be = e;
-                bz = z[j];
-            }
-        }
+        uint64_t m = best;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
-            const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
-            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-            const float oz = __shfl_xor_sync(0xffffffffu, bz, o);
-            if (better(ok, oe, bk, be)) {
-                bk = ok;
-                be = oe;
-                bz = oz;
-            }
+            const uint64_t v = shfl_xor_u64(m, o);
+            m = v > m ? v : m;
         }
+        const int be = (int)(0xFFFFFFFFu - (uint32_t)m);
+        const float bk = from_ordered((uint32_t)(m >> 32));
         if (r < k) {
-            if ((be & 31) == lane) taken |= 1u << (be >> 5);
+            sel_z[r] = __shfl_sync(0xffffffffu, best_z, be & 31);
             sel_e[r] = be;
-            sel_z[r] = bz;
             kth = bk;
+            if ((be & 31) == lane) {  // the winner's lane drops it and finds its next best
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    if (j == (be >> 5)) cand[j] = 0;
+                refresh();
+            }
         } else {
             next = bk;
         }
     }
-    double sd[kMaxTopK], sum = 0.0;
+    // w_i = s_i / sum_j s_j with s in double: lane i < k takes pick i; the sum runs in pick order
+    float my_z = 0.f;
+    int my_e = 0;
 #pragma unroll
-    for (int i = 0; i < kMaxTopK; ++i) {
-        if (i < k) {
-            sd[i] = 1.0 / (1.0 + exp(-(double)sel_z[i]));
-            sum += sd[i];
+    for (int i = 0; i < kMaxTopK; ++i)
+        if (i == lane) {
+            my_z = sel_z[i];
+            my_e = sel_e[i];
         }
-    }
+    const double sd = lane < k ? 1.0 / (1.0 + exp(-(double)my_z)) : 0.0;
+    double sum = 0.0;
 #pragma unroll
-    for (int i = 0; i < kMaxTopK; ++i) {
-        if (i < k && lane == i) {
-            idx[(int64_t)t * k + i] = sel_e[i];
-            w[(int64_t)t * k + i] = (float)(sd[i] / sum);
-        }
+    for (int i = 0; i < kMaxTopK; ++i)
+        if (i < k) sum += __shfl_sync(0xffffffffu, sd, i);
+    if (lane < k) {
+        idx[(int64_t)t * k + lane] = my_e;
+        w[(int64_t)t * k + lane] = (float)(sd / sum);
     }
     if (margin && lane == 0) margin[t] = (E > k) ? (kth - next) : INFINITY;
 }
