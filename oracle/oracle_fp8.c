@@ -90,9 +90,20 @@ void oracle_quantize_blocks(const void* x, int dt, int64_t rows, int64_t cols, i
         }
 }
 
+/* the 256 code values, filled from oracle_e4m3_decode on first use (a speed-up only) */
+static double code_value(uint8_t c) {
+    static double tab[256];
+    static int ready = 0;
+    if (!ready) {
+        for (int i = 0; i < 256; ++i) tab[i] = oracle_e4m3_decode((uint8_t)i);
+        ready = 1;
+    }
+    return tab[c];
+}
+
 /* dequantised element (r, c) of a block-quantised matrix with cols columns */
 static double deq(const uint8_t* q, const float* s, int64_t cols, int64_t blk_rows, int64_t r, int64_t c) {
-    return oracle_e4m3_decode(q[r * cols + c]) * (double)s[(r / blk_rows) * (cols / 128) + c / 128];
+    return code_value(q[r * cols + c]) * (double)s[(r / blk_rows) * (cols / 128) + c / 128];
 }
 
 /*

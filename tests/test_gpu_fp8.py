@@ -145,3 +145,30 @@ def test_fp8_forward_matches_oracle_composition(moe, name):
     ref = I["x"].double() + (wt.cpu().double().unsqueeze(-1) * yk).sum(1)
     max_abs, rel = errors(out, ref)
     assert rel < REL_L2 and max_abs < MAX_ABS, (max_abs, rel)
+
+
+def test_fp8_forward_full_decode_size_sampled(moe):
+    # the decode workload's full sizes (T=128, d=4096, E=128, d_ff=1536) through the FP8 layer; the oracle
+    # evaluates the expert MLP only for the slots of a sample of tokens
+    w = synth.WORKLOADS["decode"]
+    I = synth.make_layer_inputs(w)
+    D = {n: cuda(t) for n, t in I.items()}
+    Wq = [moe.quantize_fp8_weights(D[n]) for n in ("W_gate", "W_up", "W_down")]
+    out = torch.empty((w.T, w.d), dtype=w.out_dtype, device=DEV)
+    idx = torch.empty((w.T, 8), dtype=torch.int32, device=DEV)
+    wt = torch.empty((w.T, 8), dtype=torch.float32, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    moe.moe_forward_fp8(D["x"], D["gamma"], D["W_r"], D["b"], *Wq, out, topk_idx=idx, topk_w=wt, dev_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    tokens = [0, 1, 37, 64, 99, w.T - 1]
+    v = oracle.rmsnorm(I["x"][tokens], I["gamma"], w.eps).float()
+    vq, vs = oracle.quantize_blocks(v, 1)
+    sub_idx = idx.cpu()[tokens]
+    counts, offsets, slot_token, token_slot = oracle.permute(sub_idx, w.E)
+    Wq_cpu = [(q.cpu(), s.cpu()) for q, s in Wq]
+    r = oracle.fp8_grouped_mlp(vq[slot_token.long()], vs[slot_token.long()], counts, offsets, *Wq_cpu[0],
+                               *Wq_cpu[1], *Wq_cpu[2])
+    ref = I["x"][tokens].double() + (wt.cpu()[tokens].double().unsqueeze(-1) * r["y"][token_slot.long()]).sum(1)
+    max_abs, rel = errors(out.cpu()[tokens], ref)
+    assert rel < REL_L2 and max_abs < MAX_ABS, (max_abs, rel)
