@@ -13,6 +13,9 @@
 //                       memory; the rank of token t inside expert e's segment is
 //                       popcount(mask bits below t) + the chunk's base -> rows in
 //                       ascending token order.  Writes token_slot, slot_token.
+//   perm_single_kernel  the three above in one CTA when all tokens fit one chunk
+//                       (T <= 256, decode batches): same counts, offsets and
+//                       slots, one launch instead of three.
 //   perm_gather_kernel  16-byte chunks: each token row of v is read once and
 //                       written to its k rows of xp.
 #include "common.cuh"
@@ -124,6 +127,65 @@ __global__ void __launch_bounds__(PC) perm_scatter_kernel(const int32_t* __restr
     }
 }
 
+// T <= PC: histogram, scan over experts and scatter in one CTA (thread = token, then thread = expert)
+__global__ void __launch_bounds__(PC) perm_single_kernel(const int32_t* __restrict__ idx, int T, int E, int k,
+                                                         int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                                                         int32_t* __restrict__ slot_token,
+                                                         int32_t* __restrict__ token_slot, int32_t* status) {
+    __shared__ uint32_t mask[kMaxExperts][PC / 32];
+    __shared__ int h[kMaxExperts];
+    __shared__ int off_s[kMaxExperts];
+    __shared__ int warp_tot[PC / 32];
+    pdl_wait();
+    pdl_trigger();
+    for (int n = threadIdx.x; n < E * (PC / 32); n += PC) (&mask[0][0])[n] = 0u;
+    for (int e = threadIdx.x; e < E; e += PC) h[e] = 0;
+    __syncthreads();
+    const int t = threadIdx.x;
+    int ev[kMaxTopK];
+#pragma unroll
+    for (int i = 0; i < kMaxTopK; ++i) {
+        ev[i] = -1;
+        if (i < k && t < T) {
+            const int e = idx[(int64_t)t * k + i];
+            if (e >= 0 && e < E) {
+                ev[i] = e;
+                atomicAdd(&h[e], 1);
+                atomicOr(&mask[e][t >> 5], 1u << (t & 31));
+            } else {
+                set_status(status, DEV_BAD_EXPERT_ID);
+            }
+        }
+    }
+    __syncthreads();
+    const int e = threadIdx.x;  // PC == 256 >= E threads
+    const int cnt = e < E ? h[e] : 0;
+    const int off = block_exclusive_scan_256(cnt, warp_tot);
+    if (e < E) {
+        counts[e] = cnt;
+        offsets[e] = off;
+        off_s[e] = off;
+    }
+    if (e == PC - 1) offsets[E] = off + cnt;
+    __syncthreads();
+    if (t >= T) return;
+    const int wi = t >> 5;
+    const uint32_t below = (1u << (t & 31)) - 1u;
+#pragma unroll
+    for (int i = 0; i < kMaxTopK; ++i) {
+        if (i >= k) break;
+        const int ee = ev[i];
+        int slot = -1;
+        if (ee >= 0) {
+            int r = __popc(mask[ee][wi] & below);
+            for (int w = 0; w < wi; ++w) r += __popc(mask[ee][w]);
+            slot = off_s[ee] + r;
+            slot_token[slot] = t;
+        }
+        token_slot[(int64_t)t * k + i] = slot;
+    }
+}
+
 // each thread moves 16 bytes of one token row to the rows of its k picks
 __global__ void __launch_bounds__(256) perm_gather_kernel(const uint8_t* __restrict__ v, int64_t row_bytes,
                                                           const int32_t* __restrict__ token_slot, int T, int k,
@@ -149,6 +211,17 @@ cudaError_t launch_permute(const Ctx& c, const void* v, int v_dt, const int32_t*
                            int32_t* hist, int32_t* status) {
     const int nchunks = (T + PC - 1) / PC;
     cudaError_t err;
+    if (nchunks <= 1) {  // one chunk: the whole sort in one CTA
+        err = launch(perm_single_kernel, dim3(1), dim3(PC), 0, c, idx, T, E, k, counts, offsets, slot_token,
+                     token_slot, status);
+        if (err != cudaSuccess || T == 0 || xp == nullptr) return err;
+        const int64_t row_bytes1 = (int64_t)d * (v_dt == DT_BF16 ? 2 : 4);
+        const int64_t n1 = (int64_t)T * (row_bytes1 / 16);
+        int64_t blocks1 = (n1 + 255) / 256;
+        if (blocks1 > (int64_t)c.num_sms * 16) blocks1 = (int64_t)c.num_sms * 16;
+        return launch(perm_gather_kernel, dim3((unsigned)blocks1), dim3(256), 0, c, static_cast<const uint8_t*>(v),
+                      row_bytes1, token_slot, T, k, static_cast<uint8_t*>(xp));
+    }
     if (T > 0) {
         err = launch(perm_hist_kernel, dim3(nchunks), dim3(PC), 0, c, idx, T, E, k, hist, status);
         if (err != cudaSuccess) return err;

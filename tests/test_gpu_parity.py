@@ -103,7 +103,7 @@ def _idx(T, E, k, kind, seed):
 
 @pytest.mark.parametrize("T,E,k,kind", [(1, 16, 8, "uniform"), (255, 64, 8, "uniform"), (256, 64, 8, "uniform"),
                                         (257, 64, 8, "uniform"), (1000, 128, 8, "uniform"), (700, 256, 8, "hot"),
-                                        (513, 8, 8, "uniform"), (300, 32, 1, "uniform")])
+                                        (513, 8, 8, "uniform"), (300, 32, 1, "uniform"), (200, 256, 8, "hot")])
 @pytest.mark.parametrize("vdt", ["bf16", "f32"])
 def test_permute_bit_exact(moe, T, E, k, kind, vdt):
     d = 64
