@@ -166,3 +166,59 @@ def test_tensor_parallel_layer_equals_the_single_process_layer(world):
         assert torch.equal(r[k], r[0])
     # the d_ff split only regroups the down projection's sum; fp32 partials add fp32 rounding
     assert torch.allclose(r[0].double(), ref, rtol=1e-5, atol=1e-5)
+
+
+def _single_rank_group(port):
+    import datetime
+
+    import torch.distributed as dist
+
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=30))
+    return dist
+
+
+def _check_arguments(port, outdir):
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from moe_layer_forward_b200 import ep, tp
+
+    dist = _single_rank_group(port)
+    w, I = _inputs()
+    msgs = []
+    try:  # the rank holds fewer experts than E / N
+        ep.ep_forward(I["x"], I["gamma"], I["W_r"], I["b"], I["W_gate"][:3], I["W_up"][:3], I["W_down"][:3], E=w.E,
+                      ops=OracleOps())
+    except ValueError as e:
+        msgs.append(str(e))
+    try:  # the down slice does not match the gate/up feature slice
+        tp.tp_forward(I["x"], I["gamma"], I["W_r"], I["b"], I["W_gate"], I["W_up"], I["W_down"][:, :, :64],
+                      ops=OracleOps())
+    except ValueError as e:
+        msgs.append(str(e))
+    # one rank: both orchestrations reduce to the plain layer
+    out, stats = ep.ep_forward(I["x"], I["gamma"], I["W_r"], I["b"], I["W_gate"], I["W_up"], I["W_down"], E=w.E,
+                               top_k=w.top_k, eps=w.eps, ops=OracleOps())
+    out_tp = tp.tp_forward(I["x"], I["gamma"], I["W_r"], I["b"], I["W_gate"], I["W_up"], I["W_down"], top_k=w.top_k,
+                           eps=w.eps, ops=OracleOps())
+    torch.save({"msgs": msgs, "out": out, "out_tp": out_tp, "rows": stats.rows_received},
+               os.path.join(outdir, "r.pt"))
+    dist.destroy_process_group()
+
+
+def test_orchestration_argument_checks_and_single_rank():
+    w, I = _inputs()
+    with tempfile.TemporaryDirectory() as d:
+        _spawn_one(_check_arguments, d)
+        r = torch.load(os.path.join(d, "r.pt"))
+    assert len(r["msgs"]) == 2 and "experts" in r["msgs"][0] and "slice" in r["msgs"][1]
+    assert r["rows"] == w.T * w.top_k
+    assert torch.allclose(r["out"].double(), r["out_tp"].double(), rtol=1e-6, atol=1e-6)
+
+
+def _one(rank, fn, port, outdir):
+    fn(port, outdir)
+
+
+def _spawn_one(fn, outdir):
+    mp.start_processes(_one, args=(fn, _free_port(), outdir), nprocs=1, join=True, start_method="spawn")
