@@ -12,7 +12,8 @@
 //   quant_rows_kernel      a warp per (row, 128-column block) of a GEMM input
 //   quant_tiles_kernel     a CTA per 128 x 128 block of a weight matrix
 //   rmsnorm_quant_kernel   RMSNorm of a row (the same fp32 arithmetic as the bf16
-//                          path) quantised per 128 columns, plus 1/rms for the router
+//                          path) quantised per 128 columns, plus 1/rms for the router;
+//                          rmsnorm_quant_row_kernel the same with a CTA per row (few rows)
 //   grouped_gemm_fp8_kernel<SWIGLU, R>
 //       weights are the MMA's M operand: 128 weight rows = one row of scale blocks;
 //       the expert's rows (tokens) are N <= R.  K runs in 128-wide blocks: a stage
@@ -160,6 +161,50 @@ __global__ void __launch_bounds__(256) rmsnorm_quant_kernel(const void* __restri
     if (lane == 0) rstd_out[t] = r;
     const int nb = d / 128;
     for (int b = 0; b < nb; ++b) {
+        const int j = b * 128 + 4 * lane;
+        float a[4], g[4], v[4], sc;
+        load4<XDT>(x, row + j, a);
+        load4<DT_F32>(gamma, j, g);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = (a[i] * r) * g[i];
+        const uint32_t codes = quant_block4(v, sc);
+        *reinterpret_cast<uint32_t*>(q + row + j) = codes;
+        if (lane == 0) s[t * nb + b] = sc;
+    }
+}
+
+// The same for batches of fewer rows than two waves of warp-per-row CTAs: a
+// 256-thread CTA per row sums the squares in the order of the bf16 path's
+// row kernel (so 1/rms is the same to the bit), then each warp quantises
+// 128-column blocks w, w + 8, ... of the row.
+template <int XDT>
+__global__ void __launch_bounds__(256) rmsnorm_quant_row_kernel(const void* __restrict__ x,
+                                                                const float* __restrict__ gamma, int T, int d,
+                                                                float eps, uint8_t* __restrict__ q,
+                                                                float* __restrict__ s, float* __restrict__ rstd_out) {
+    __shared__ float part[8];
+    pdl_wait();
+    pdl_trigger();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t = blockIdx.x, row = t * d;
+    float ss = 0.f;
+    for (int j = threadIdx.x * 8; j < d; j += 2048) {
+        float a[8];
+        load8<XDT>(x, row + j, a);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ss = fmaf(a[i], a[i], ss);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane == 0) part[warp] = ss;
+    __syncthreads();
+    ss = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) ss += part[w];
+    const float r = 1.0f / sqrtf(ss / (float)d + eps);
+    if (threadIdx.x == 0) rstd_out[t] = r;
+    const int nb = d / 128;
+    for (int b = warp; b < nb; b += 8) {
         const int j = b * 128 + 4 * lane;
         float a[4], g[4], v[4], sc;
         load4<XDT>(x, row + j, a);
@@ -582,6 +627,12 @@ cudaError_t launch_quant_fp8(const Ctx& c, const void* x, int dt, int64_t rows, 
 cudaError_t launch_rmsnorm_quant(const Ctx& c, const void* x, int x_dt, const float* gamma, int T, int d, float eps,
                                  uint8_t* q, float* s, float* rstd) {
     if (T == 0) return cudaSuccess;
+    if (T <= 2 * 8 * c.num_sms) {  // fewer rows than two waves of warp-per-row CTAs
+        if (x_dt == DT_BF16)
+            return launch(fp8::rmsnorm_quant_row_kernel<DT_BF16>, dim3(T), dim3(256), 0, c, x, gamma, T, d, eps, q, s,
+                          rstd);
+        return launch(fp8::rmsnorm_quant_row_kernel<DT_F32>, dim3(T), dim3(256), 0, c, x, gamma, T, d, eps, q, s, rstd);
+    }
     const dim3 g((T + 7) / 8);
     if (x_dt == DT_BF16) return launch(fp8::rmsnorm_quant_kernel<DT_BF16>, g, dim3(256), 0, c, x, gamma, T, d, eps, q, s, rstd);
     return launch(fp8::rmsnorm_quant_kernel<DT_F32>, g, dim3(256), 0, c, x, gamma, T, d, eps, q, s, rstd);
