@@ -14,9 +14,12 @@
 //   rmsnorm_quant_kernel   RMSNorm of a row (the same fp32 arithmetic as the bf16
 //                          path) quantised per 128 columns, plus 1/rms for the router;
 //                          rmsnorm_quant_row_kernel the same with a CTA per row (few rows)
-//   grouped_gemm_fp8_kernel<SWIGLU, R>
+//   grouped_gemm_fp8_kernel<SWIGLU, R, NA>
 //       weights are the MMA's M operand: 128 weight rows = one row of scale blocks;
-//       the expert's rows (tokens) are N <= R.  K runs in 128-wide blocks: a stage
+//       the expert's rows (tokens) are N <= R.  A tile stages NA = 2 such operands
+//       (gate and up, or two consecutive 128-feature blocks of down), because the
+//       promotion pass below, not the MMAs or the loads, sets the pace: two
+//       operands bring 32 KB of weights per pass.  K runs in 128-wide blocks: a stage
 //       holds one 128-byte swizzled row slice per operand (exactly one scale block),
 //       and the MMA thread issues 4 kind::f8f6f4 MMAs (K = 32) per operand into one
 //       of eight tensor-memory chunk buffers.  Four epilogue warps promote each chunk
@@ -221,10 +224,14 @@ __global__ void __launch_bounds__(256) rmsnorm_quant_row_kernel(const void* __re
 constexpr int kThreads = 320;
 constexpr int kSmemLimit = 232448;
 
-template <bool SWIGLU, int R>
+// NA = 128-row weight operands per tile: gate/up stages a gate and an up block
+// (NA = 2); down stages one (128 output features) or two consecutive ones (256).
+template <bool SWIGLU, int R, int NA>
 struct Cfg {
     static_assert(R == 16 || R == 32, "token columns per tile");
-    static constexpr int NUM_A = SWIGLU ? 2 : 1;
+    static_assert(NA == 2 || (!SWIGLU && NA == 1), "weight operands per tile");
+    static constexpr int NUM_A = NA;
+    static constexpr int WROWS = SWIGLU ? 128 : 128 * NA;  // output features of a tile
     static constexpr int A_BYTES = 128 * 128;  // 128 weight rows x one 128-byte K block
     static constexpr int B_BYTES = R * 128;
     static constexpr int STAGE_BYTES = NUM_A * A_BYTES + B_BYTES;
@@ -232,7 +239,7 @@ struct Cfg {
     static constexpr int STAGES_MAX = (kSmemLimit - 1024 - AUX_BYTES) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_MAX > 8 ? 8 : STAGES_MAX;
     static_assert(STAGES >= 3, "pipeline depth");
-    static constexpr int CB = NUM_A * R;  // columns of one chunk buffer: gate | up
+    static constexpr int CB = NUM_A * R;  // columns of one chunk buffer: gate | up, or the two down blocks
     static constexpr int NBUF = 8;        // chunk buffers: the MMAs run up to 7 K blocks ahead of the promotion
     static constexpr int TMEM_COLS = NBUF * CB <= 128 ? 128 : (NBUF * CB <= 256 ? 256 : 512);
     static_assert(NBUF * CB <= 512, "tensor memory");
@@ -285,11 +292,11 @@ __device__ __forceinline__ void decode_tile(const Aux& a, int E, int R, int tile
     rb = local - cb * nrb;
 }
 
-template <bool SWIGLU, int R>
+template <bool SWIGLU, int R, int NA>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tm_w1, const __grid_constant__ CUtensorMap tm_w2,
                             const Args p) {
-    using C = Cfg<SWIGLU, R>;
+    using C = Cfg<SWIGLU, R, NA>;
     constexpr int STAGES = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -323,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncthreads();
     if (warp == 0) {
-        const int ncb = p.n_out / 128;
+        const int ncb = p.n_out / C::WROWS;
         int loc[8], sum = 0;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -368,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
             int e, rb, cb;
             decode_tile(aux, E, R, tile, e, rb, cb);
-            const int w_row = e * p.n_out + cb * 128;
+            const int w_row = e * p.n_out + cb * C::WROWS;
             bool ok = true;
             for (int kb = 0; kb < nk; ++kb) {
                 const uint32_t full = smem_u32(&aux.full[stage]);
@@ -382,6 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_expect_tx(full, C::NUM_A * C::A_BYTES);
                     tma_load_2d(a0, &tm_w1, kb * 128, w_row, full);
                     if (SWIGLU) tma_load_2d(a0 + C::A_BYTES, &tm_w2, kb * 128, w_row, full);
+                    else if (NA == 2) tma_load_2d(a0 + C::A_BYTES, &tm_w1, kb * 128, w_row + 128, full);
                 }
                 used |= 1u << stage;
                 last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
@@ -421,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint64_t bd = sdesc_sw128(b0 + kk * 32);
                         tc_mma_f8(d, sdesc_sw128(a0 + kk * 32), bd, idesc, kk > 0 ? 1u : 0u);
-                        if (SWIGLU) tc_mma_f8(d + R, sdesc_sw128(a0 + C::A_BYTES + kk * 32), bd, idesc, kk > 0 ? 1u : 0u);
+                        if (NA == 2) tc_mma_f8(d + R, sdesc_sw128(a0 + C::A_BYTES + kk * 32), bd, idesc, kk > 0 ? 1u : 0u);
                     }
                     tc_commit(smem_u32(&aux.empty[stage]));
                     tc_commit(smem_u32(&aux.cfull[c]));
@@ -493,19 +501,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int base = aux.off[e] + rb * R;
             // lane n < rows: input row of token column n (its activation scales)
             const int my_row = lane < rows ? (p.gather ? p.gather[base + lane] : base + lane) : 0;
-            const float* s1 = p.w1_s + ((int64_t)e * (p.n_out / 128) + cb) * nk;
-            const float* s2 = SWIGLU ? p.w2_s + ((int64_t)e * (p.n_out / 128) + cb) * nk : nullptr;
+            // weight scale rows: gate and up of block cb, or down blocks NA*cb (and NA*cb + 1)
+            const int64_t wb = (int64_t)e * (p.n_out / 128) + (SWIGLU ? cb : NA * cb);
+            const float* s1 = p.w1_s + wb * nk;
+            const float* s2 = SWIGLU ? p.w2_s + wb * nk : (NA == 2 ? p.w1_s + (wb + 1) * nk : nullptr);
             float g[R], u[R];
 #pragma unroll
             for (int n = 0; n < R; ++n) g[n] = u[n] = 0.f;
             // scales of the next block load while this block's chunk is awaited
-            float sw1_n = __ldg(s1), sw2_n = SWIGLU ? __ldg(s2) : 0.f;
+            float sw1_n = __ldg(s1), sw2_n = NA == 2 ? __ldg(s2) : 0.f;
             float sa_n = lane < rows ? __ldg(p.act_s + (int64_t)my_row * nk) : 0.f;
             for (int kb = 0; kb < nk; ++kb, ++q) {
                 const float sw1 = sw1_n, sw2 = sw2_n, my_sa = sa_n;
                 if (kb + 1 < nk) {
                     sw1_n = __ldg(s1 + kb + 1);
-                    if (SWIGLU) sw2_n = __ldg(s2 + kb + 1);
+                    if (NA == 2) sw2_n = __ldg(s2 + kb + 1);
                     sa_n = lane < rows ? __ldg(p.act_s + (int64_t)my_row * nk + kb + 1) : 0.f;
                 }
                 const uint32_t c = q % C::NBUF, use = q / C::NBUF;
@@ -518,9 +528,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t ta = tmem_base + c * C::CB + ((uint32_t)(32 * qw) << 16);
                 uint32_t cg[R], cu[R];
                 tmem_ld<R>(ta, cg);
-                if (SWIGLU) tmem_ld<R>(ta + R, cu);
+                if (NA == 2) tmem_ld<R>(ta + R, cu);
                 tmem_wait_ld(cg);
-                if (SWIGLU) tmem_wait_ld(cu);
+                if (NA == 2) tmem_wait_ld(cu);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&aux.cempty[c]));
@@ -528,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int n = 0; n < R; ++n) {
                     const float sa = __shfl_sync(0xffffffffu, my_sa, n);
                     g[n] = fmaf(__uint_as_float(cg[n]), sw1 * sa, g[n]);
-                    if (SWIGLU) u[n] = fmaf(__uint_as_float(cu[n]), sw2 * sa, u[n]);
+                    if (NA == 2) u[n] = fmaf(__uint_as_float(cu[n]), sw2 * sa, u[n]);
                 }
             }
             if (!ok) break;
@@ -562,7 +572,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
 #pragma unroll
                 for (int n = 0; n < R; ++n)
-                    if (n < rows) p.out[(int64_t)(base + n) * p.n_out + cb * 128 + f] = (uint16_t)f32_to_bf16_bits(g[n]);
+                    if (n < rows) {
+                        uint16_t* o = p.out + (int64_t)(base + n) * p.n_out + cb * C::WROWS + f;
+                        o[0] = (uint16_t)f32_to_bf16_bits(g[n]);
+                        if (NA == 2) o[128] = (uint16_t)f32_to_bf16_bits(u[n]);
+                    }
             }
         }
     }
@@ -586,10 +600,10 @@ static bool encode_u8(CUtensorMap* tm, const void* base, uint64_t inner, uint64_
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool SWIGLU, int R>
+template <bool SWIGLU, int R, int NA = 2>
 static cudaError_t run(const Ctx& c, int S, const void* w1, const void* w2, const Args& a) {
-    using CF = Cfg<SWIGLU, R>;
-    auto kern = grouped_gemm_fp8_kernel<SWIGLU, R>;
+    using CF = Cfg<SWIGLU, R, NA>;
+    auto kern = grouped_gemm_fp8_kernel<SWIGLU, R, NA>;
     static bool attr_done[64] = {};
     if (c.device < 0 || c.device >= 64) return cudaErrorInvalidDevice;
     if (!attr_done[c.device]) {
@@ -601,7 +615,7 @@ static cudaError_t run(const Ctx& c, int S, const void* w1, const void* w2, cons
     const uint64_t wrows = (uint64_t)a.E * a.n_out;
     if (!encode_u8(&tm_w1, w1, (uint64_t)a.K, wrows)) return cudaErrorInvalidValue;
     if (!encode_u8(&tm_w2, SWIGLU ? w2 : w1, (uint64_t)a.K, wrows)) return cudaErrorInvalidValue;
-    const int64_t max_tiles = ((int64_t)S / R + a.E) * (a.n_out / 128);
+    const int64_t max_tiles = ((int64_t)S / R + a.E) * (a.n_out / CF::WROWS);
     const int grid = (int)(max_tiles < c.num_sms ? max_tiles : c.num_sms);
     if (grid <= 0) return cudaSuccess;
     return launch(kern, dim3(grid), dim3(kThreads), (size_t)CF::SMEM, c, tm_w1, tm_w2, a);
@@ -657,8 +671,12 @@ cudaError_t launch_down_fp8(const Ctx& c, const uint8_t* hq, const float* hs, co
     if (S == 0) return cudaSuccess;
     fp8::Args a{counts, offsets, E, d_ff, d, hq, hs, nullptr, Wd_s, nullptr, nullptr, nullptr,
                 static_cast<uint16_t*>(y), status};
-    if (fp8_rows(S, E) == 16) return fp8::run<false, 16>(c, S, Wd, nullptr, a);
-    return fp8::run<false, 32>(c, S, Wd, nullptr, a);
+    // two 128-row weight blocks per tile where d allows: each promotion pass then covers 32 KB of
+    // weights instead of 16 (the pass, not the MMAs or the loads, paces the 128-row tile)
+    const bool wide = d % 256 == 0;
+    if (fp8_rows(S, E) == 16)
+        return wide ? fp8::run<false, 16, 2>(c, S, Wd, nullptr, a) : fp8::run<false, 16, 1>(c, S, Wd, nullptr, a);
+    return wide ? fp8::run<false, 32, 2>(c, S, Wd, nullptr, a) : fp8::run<false, 32, 1>(c, S, Wd, nullptr, a);
 }
 
 }  // namespace moe

@@ -77,7 +77,7 @@ def _expert_inputs(counts, d, d_ff, seed):
 
 
 @pytest.mark.parametrize("case", list(COUNTS))
-@pytest.mark.parametrize("d,d_ff", [(256, 256), (512, 384)])
+@pytest.mark.parametrize("d,d_ff", [(256, 256), (512, 384), (384, 256)])  # down tiles of 256 / 256 / 128 features
 def test_fp8_grouped_swiglu_matches_oracle(moe, case, d, d_ff):
     counts = COUNTS[case]
     ct, offs, xq, xs, Wq = _expert_inputs(counts, d, d_ff, seed=810)
