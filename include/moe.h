@@ -133,6 +133,8 @@ moe_status_t moe_router_topk(const void* v, moe_dtype_t v_dt, const float* W_r, 
  *   xp[r][:]       = v[slot_token[r]][:]   (dtype v_dt)
  * Rows inside a segment follow ascending token index, so the result is
  * deterministic.  Bad ids set MOE_DEV_BAD_EXPERT_ID and are dropped.
+ * xp may be NULL: then only the maps are written (moe_ep_dispatch moves the
+ * rows itself).
  * Requires d % 8 == 0, v and xp 16-byte aligned, 1 <= k <= 8, k <= E <= 256.
  */
 moe_status_t moe_permute(const void* v, moe_dtype_t v_dt, const int32_t* topk_idx, int32_t T, int32_t d, int32_t E,
@@ -291,6 +293,53 @@ moe_status_t moe_grouped_swiglu_fp8(const uint8_t* xq, const float* xs, const mo
 moe_status_t moe_forward_fp8(const moe_shape_t* shape, const moe_weights_fp8_t* w, const void* x, void* out,
                              int32_t* topk_idx, float* topk_w, float* logits, void* ws, size_t* ws_bytes,
                              int32_t* dev_status, moe_stream_t stream);
+
+/*
+ * Expert parallelism over peer memory (steps 3 and 5 fused with their
+ * exchanges) [P5 §Token 分发策略: every (token, expert) row goes to the rank
+ * that owns the expert and the results are summed back at the token's source;
+ * P1 §EP 路径: the same exchange around the grouped GEMM].
+ *
+ * N ranks (one GPU each); rank j owns experts [j E/N, (j+1) E/N).  Every rank
+ * first runs steps 1-3 on its own tokens (moe_permute with xp = NULL), then the
+ * ranks exchange their counts so that each holds the same count_table
+ * [N][E] (int32, device): count_table[s][e] = rows rank s routes to expert e.
+ * Rank j's receive buffer then holds its experts' rows expert-major, within an
+ * expert by source rank, within a source in that source's slot order:
+ *   row(source r, expert e, i) = sum_{e' in [j E/N, e)} sum_s count_table[s][e']
+ *                                + sum_{s < r} count_table[s][e] + i
+ * which is the layout moe_grouped_swiglu takes, with counts and offsets from
+ * moe_ep_layout.  recv_bufs / y_bufs are device arrays of N device pointers:
+ * entry j is rank j's receive buffer / expert output buffer ([rows][d], dtype
+ * of v / y, 16-byte aligned), mapped into this process (NVLink peer access or
+ * the same GPU).  The calls only load and store through them: the caller
+ * orders the ranks (all dispatches complete before any rank's expert MLP reads
+ * its receive buffer; all expert MLPs complete before any combine reads their
+ * outputs).  Requires E % N == 0, N <= MOE_MAX_EP_RANKS, d % 8 == 0.
+ *
+ * moe_ep_dispatch: the permutation's row copy to the owners: for every pick
+ *   (t, i) of this rank with expert e = topk_idx[t][i] and slot
+ *   s = token_slot[t][i], recv_bufs[e / (E/N)][row(rank, e, s - offsets[e])] = v[t].
+ *   topk_idx / token_slot / offsets as returned by moe_router_topk and
+ *   moe_permute on this rank.  A bad pick sets MOE_DEV_BAD_EXPERT_ID.
+ * moe_ep_layout: counts_loc[e] = sum_s count_table[s][rank E/N + e] and
+ *   offsets_loc[0 .. E/N] its exclusive prefix (the receive buffer's segments).
+ * moe_ep_combine: step 5 with each pick's expert output row read from its
+ *   owner: out[t] = residual[t] + sum_{i<k} topk_w[t][i] * y_bufs[owner][row]
+ *   in fp32, pick order; the same arithmetic as moe_unpermute_combine.
+ */
+#define MOE_MAX_EP_RANKS 64
+moe_status_t moe_ep_dispatch(const void* v, moe_dtype_t v_dt, const int32_t* topk_idx, const int32_t* token_slot,
+                             const int32_t* offsets, const int32_t* count_table, int32_t rank, int32_t N, int32_t E,
+                             int32_t T, int32_t d, int32_t k, void* const* recv_bufs, int32_t* dev_status,
+                             moe_stream_t stream);
+moe_status_t moe_ep_layout(const int32_t* count_table, int32_t rank, int32_t N, int32_t E, int32_t* counts_loc,
+                           int32_t* offsets_loc, moe_stream_t stream);
+moe_status_t moe_ep_combine(const void* const* y_bufs, moe_dtype_t y_dt, const int32_t* topk_idx,
+                            const int32_t* token_slot, const int32_t* offsets, const int32_t* count_table,
+                            int32_t rank, int32_t N, int32_t E, const float* topk_w, const void* residual,
+                            moe_dtype_t r_dt, int32_t T, int32_t d, int32_t k, void* out, moe_dtype_t out_dt,
+                            int32_t* dev_status, moe_stream_t stream);
 
 /* Number of kernels the library has enqueued in this process since it was
  * loaded, over all entry points, streams and threads (successful launches

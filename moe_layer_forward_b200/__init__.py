@@ -62,6 +62,10 @@ _sig = {
                                _vp, _vp, _vp],
     "moe_forward_fp8": [ctypes.POINTER(MoeShape), ctypes.POINTER(MoeWeightsFP8), _vp, _vp, _vp, _vp, _vp, _vp, _szp,
                         _vp, _vp],
+    "moe_ep_dispatch": [_vp, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp],
+    "moe_ep_layout": [_vp, _i32, _i32, _i32, _vp, _vp, _vp],
+    "moe_ep_combine": [_vp, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _i32,
+                       _vp, _vp],
 }
 for _name, _args in _sig.items():
     _fn = getattr(_lib, _name)
@@ -207,6 +211,42 @@ def moe_unpermute_combine(y, token_slot, topk_w, residual, out) -> None:
     _check("moe_unpermute_combine", _lib.moe_unpermute_combine(_p(y), _dt(y), _p(token_slot), _p(topk_w),
                                                                _p(residual), _dt(residual), T, d, k, _p(out),
                                                                _dt(out), _stream(residual.device)))
+
+
+# --------------------------------------------------------------------------- expert parallelism over peer memory
+def moe_ep_dispatch(v, topk_idx, token_slot, offsets, count_table, rank: int, recv_ptrs, dev_status=None) -> None:
+    """Store this rank's routed rows of v into their owners' receive buffers.
+
+    count_table: int32 [N][E] on the device (every rank's counts); recv_ptrs: int64 [N] on the device, the
+    receive buffers' addresses as mapped into this process."""
+    T, d = v.shape
+    k = topk_idx.shape[1]
+    N, E = count_table.shape
+    _check("moe_ep_dispatch", _lib.moe_ep_dispatch(_p(v), _dt(v), _p(topk_idx), _p(token_slot), _p(offsets),
+                                                   _p(count_table), rank, N, E, T, d, k, _p(recv_ptrs),
+                                                   _p(dev_status), _stream(v.device)))
+
+
+def moe_ep_layout(count_table, rank: int, counts_loc, offsets_loc) -> None:
+    """This rank's expert segments of its receive buffer: counts_loc [E/N], offsets_loc [E/N + 1]."""
+    N, E = count_table.shape
+    _check("moe_ep_layout", _lib.moe_ep_layout(_p(count_table), rank, N, E, _p(counts_loc), _p(offsets_loc),
+                                               _stream(count_table.device)))
+
+
+def moe_ep_combine(y_ptrs, y_dtype, topk_idx, token_slot, offsets, count_table, rank: int, topk_w, residual, out,
+                   dev_status=None) -> None:
+    """out = residual + sum_i w_i y_i with each pick's row y_i read from its owner's output buffer.
+
+    y_ptrs: int64 [N] on the device, the expert output buffers' addresses; y_dtype their torch dtype."""
+    T, d = residual.shape
+    k = topk_idx.shape[1]
+    N, E = count_table.shape
+    ydt = MOE_BF16 if y_dtype == torch.bfloat16 else MOE_F32
+    _check("moe_ep_combine", _lib.moe_ep_combine(_p(y_ptrs), ydt, _p(topk_idx), _p(token_slot), _p(offsets),
+                                                 _p(count_table), rank, N, E, _p(topk_w), _p(residual),
+                                                 _dt(residual), T, d, k, _p(out), _dt(out), _p(dev_status),
+                                                 _stream(residual.device)))
 
 
 def _shape(x, W_gate, out, top_k, eps, E) -> MoeShape:

@@ -175,7 +175,8 @@ moe_status_t moe_permute(const void* v, moe_dtype_t v_dt, const int32_t* topk_id
     st = check_ws(ws, ws_bytes, cv.off, &query);
     if (st != MOE_OK || query) return st;
     if (!counts || !offsets) return MOE_ERR_INVALID_ARG;
-    if (T > 0 && (!v || !topk_idx || !slot_token || !token_slot || !xp || !aligned16(v) || !aligned16(xp)))
+    // xp == NULL: the maps only (a caller that moves the rows itself, e.g. moe_ep_dispatch)
+    if (T > 0 && (!v || !topk_idx || !slot_token || !token_slot || !aligned16(v) || (xp && !aligned16(xp))))
         return MOE_ERR_INVALID_ARG;
     Ctx c;
     st = make_ctx(stream, c);
@@ -265,6 +266,61 @@ moe_status_t moe_unpermute_combine(const void* y, moe_dtype_t y_dt, const int32_
     moe_status_t st = make_ctx(stream, c);
     if (st != MOE_OK) return st;
     return cuda_status(launch_combine(c, y, y_dt, token_slot, topk_w, residual, r_dt, T, d, k, out, out_dt));
+}
+
+// ----------------------------------------------------------------------------- expert parallelism over peer memory
+namespace {
+moe_status_t check_ep(int32_t rank, int32_t N, int32_t E, int32_t T, int32_t d, int32_t k, const int32_t* table) {
+    if (N <= 0 || rank < 0 || rank >= N || E <= 0 || T < 0 || d <= 0 || k <= 0 || !table) return MOE_ERR_INVALID_ARG;
+    if (E % N != 0 || E > MOE_MAX_EXPERTS || k > MOE_MAX_TOP_K || d % 8 != 0 || N > MOE_MAX_EP_RANKS)
+        return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+}  // namespace
+
+moe_status_t moe_ep_dispatch(const void* v, moe_dtype_t v_dt, const int32_t* topk_idx, const int32_t* token_slot,
+                             const int32_t* offsets, const int32_t* count_table, int32_t rank, int32_t N, int32_t E,
+                             int32_t T, int32_t d, int32_t k, void* const* recv_bufs, int32_t* dev_status,
+                             moe_stream_t stream) {
+    if (!valid_dt(v_dt)) return MOE_ERR_INVALID_ARG;
+    moe_status_t st = check_ep(rank, N, E, T, d, k, count_table);
+    if (st != MOE_OK) return st;
+    if (T == 0) return MOE_OK;
+    if (!v || !topk_idx || !token_slot || !offsets || !recv_bufs || !aligned16(v)) return MOE_ERR_INVALID_ARG;
+    Ctx c;
+    st = make_ctx(stream, c);
+    if (st != MOE_OK) return st;
+    return cuda_status(launch_ep_dispatch(c, v, v_dt, topk_idx, token_slot, offsets, count_table, rank, N, E, T, d, k,
+                                          recv_bufs, dev_status));
+}
+
+moe_status_t moe_ep_layout(const int32_t* count_table, int32_t rank, int32_t N, int32_t E, int32_t* counts_loc,
+                           int32_t* offsets_loc, moe_stream_t stream) {
+    moe_status_t st = check_ep(rank, N, E, 0, 8, 1, count_table);
+    if (st != MOE_OK) return st;
+    if (!counts_loc || !offsets_loc) return MOE_ERR_INVALID_ARG;
+    Ctx c;
+    st = make_ctx(stream, c);
+    if (st != MOE_OK) return st;
+    return cuda_status(launch_ep_layout(c, count_table, rank, N, E, counts_loc, offsets_loc));
+}
+
+moe_status_t moe_ep_combine(const void* const* y_bufs, moe_dtype_t y_dt, const int32_t* topk_idx,
+                            const int32_t* token_slot, const int32_t* offsets, const int32_t* count_table,
+                            int32_t rank, int32_t N, int32_t E, const float* topk_w, const void* residual,
+                            moe_dtype_t r_dt, int32_t T, int32_t d, int32_t k, void* out, moe_dtype_t out_dt,
+                            int32_t* dev_status, moe_stream_t stream) {
+    if (!valid_dt(y_dt) || !valid_dt(r_dt) || !valid_dt(out_dt)) return MOE_ERR_INVALID_ARG;
+    moe_status_t st = check_ep(rank, N, E, T, d, k, count_table);
+    if (st != MOE_OK) return st;
+    if (T == 0) return MOE_OK;
+    if (!y_bufs || !topk_idx || !token_slot || !offsets || !topk_w || !residual || !out) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(residual) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+    Ctx c;
+    st = make_ctx(stream, c);
+    if (st != MOE_OK) return st;
+    return cuda_status(launch_ep_combine(c, y_bufs, y_dt, topk_idx, token_slot, offsets, count_table, rank, N, E,
+                                         topk_w, residual, r_dt, T, d, k, out, out_dt, dev_status));
 }
 
 moe_status_t moe_forward(const moe_shape_t* shape, const moe_weights_t* wts, const void* x, void* out,

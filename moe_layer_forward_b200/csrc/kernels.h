@@ -70,6 +70,18 @@ cudaError_t launch_permute(const Ctx& c, const void* v, int v_dt, const int32_t*
                            int32_t* counts, int32_t* offsets, int32_t* slot_token, int32_t* token_slot, void* xp,
                            int32_t* hist, int32_t* status);
 
+// ---- steps 3 and 5 with expert parallelism over peer memory (ep_p2p.cu)
+// table [N][E]: rows every rank routes to every expert; recv / y: device arrays of N peer pointers
+cudaError_t launch_ep_dispatch(const Ctx& c, const void* v, int v_dt, const int32_t* idx, const int32_t* token_slot,
+                               const int32_t* offsets, const int32_t* table, int rank, int N, int E, int T, int d,
+                               int k, void* const* recv, int32_t* status);
+cudaError_t launch_ep_layout(const Ctx& c, const int32_t* table, int rank, int N, int E, int32_t* counts_loc,
+                             int32_t* offsets_loc);
+cudaError_t launch_ep_combine(const Ctx& c, const void* const* y, int y_dt, const int32_t* idx,
+                              const int32_t* token_slot, const int32_t* offsets, const int32_t* table, int rank, int N,
+                              int E, const float* w, const void* res, int r_dt, int T, int d, int k, void* out,
+                              int out_dt, int32_t* status);
+
 // ---- step 4: expert MLP (expert_tc.cu: bf16 tensor cores; expert_simt.cu: fp32)
 // gate/up: xp holds the S permuted rows; or, with gather, xp holds act_rows rows and slot i
 // reads row gather[i] (the permutation's slot -> token map), so no permuted copy is made.
