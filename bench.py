@@ -46,6 +46,7 @@ def parse():
                          "for ncu captures of the same kernels, never for reported numbers")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-ep", action="store_true", help="skip the one-rank expert-parallel (peer memory) timing")
     ap.add_argument("--no-fp8", action="store_true",
                     help="skip the block-FP8 layer timing (run for bf16 workloads of <= 32 rows per expert)")
     ap.add_argument("--no-masked", action="store_true",
@@ -391,6 +392,33 @@ def run_ours(a, w):
                "vs_bf16_layer": ms_per_step / fms}
         del Wq
 
+    # ---- expert parallelism with the exchange fused into the dispatch and combine kernels: one rank's step
+    epp = None
+    if not a.no_ep and world == 1 and w.w_dtype == torch.bfloat16:
+        from moe_layer_forward_b200 import ep_p2p
+
+        peers = ep_p2p.local_peers(1, ep_p2p.capacity_rows(T, 1, k, E), w.d, w.w_dtype, dev)
+
+        def estep():
+            return ep_p2p.ep_p2p_forward_emulated([D["x"]], D["gamma"], D["W_r"], D["b"], D["W_gate"], D["W_up"],
+                                                  D["W_down"], top_k=k, eps=w.eps, peers=peers)
+
+        for _ in range(a.warmup):
+            estep()
+        barrier()
+        p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        p0.record()
+        for _ in range(a.steps):
+            estep()
+        p1.record()
+        torch.cuda.synchronize()
+        ems = p0.elapsed_time(p1) / a.steps
+        epp = {"ranks": 1, "ms_per_step": ems, "tokens_per_s": T / (ems / 1000.0), "vs_moe_forward": ms_per_step / ems,
+               "steps": "routing, permutation maps, dispatch into the receive buffer, layout, grouped MLP over "
+                        "the whole buffer, pull combine; no host synchronisation",
+               "multi_gpu": "not measured (one GPU per call here)"}
+        del peers
+
     # ---- end to end through the public API with host buffers
     e2e = None
     if not a.no_e2e:
@@ -427,7 +455,8 @@ def run_ours(a, w):
                 "vs_baseline": None, "dtype": "bf16" if w.w_dtype == torch.bfloat16 else "f32",
                 "data": "synthetic", "config": config_of(w, world), "roofline": roof, "cpu_baseline": cpu,
                 "e2e": e2e, "gpu_launches": launches, "clocks": clk.summary(),
-                "stages_ms": stage_ms, "active_experts": active, "masked_layout": masked, "fp8_layer": fp8}
+                "stages_ms": stage_ms, "active_experts": active, "masked_layout": masked, "fp8_layer": fp8,
+                "ep_p2p": epp}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

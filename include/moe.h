@@ -201,6 +201,19 @@ moe_status_t moe_grouped_swiglu(const void* xp, const void* W_gate, const void* 
                                 int32_t d, int32_t d_ff, void* h, void* y, int32_t* dev_status, moe_stream_t stream);
 
 /*
+ * Step 4 for a caller that knows its buffer size but not its row count on the
+ * host [same computation as moe_grouped_swiglu]: xp, h, y hold S_cap rows;
+ * counts/offsets (device) decide which rows are computed, and the tile form is
+ * chosen as if there were S_expected rows (1 <= S_expected <= S_cap), so the
+ * call needs no device-to-host read.  With S_expected == S_cap it is
+ * moe_grouped_swiglu.  Rows outside every segment are not written.
+ */
+moe_status_t moe_grouped_swiglu_sized(const void* xp, const void* W_gate, const void* W_up, const void* W_down,
+                                      moe_dtype_t dt, const int32_t* counts, const int32_t* offsets, int32_t S_cap,
+                                      int32_t S_expected, int32_t E, int32_t d, int32_t d_ff, void* h, void* y,
+                                      int32_t* dev_status, moe_stream_t stream);
+
+/*
  * Step 4 on the masked decode layout [P5 §专家计算实现: deepgemm_masked, the
  * decode-phase expert GEMM; the page names it without defining it, and this
  * follows the reading that its input is per-expert buffers of fixed capacity

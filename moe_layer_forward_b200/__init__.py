@@ -62,6 +62,8 @@ _sig = {
                                _vp, _vp, _vp],
     "moe_forward_fp8": [ctypes.POINTER(MoeShape), ctypes.POINTER(MoeWeightsFP8), _vp, _vp, _vp, _vp, _vp, _vp, _szp,
                         _vp, _vp],
+    "moe_grouped_swiglu_sized": [_vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp,
+                                 _vp],
     "moe_ep_dispatch": [_vp, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp],
     "moe_ep_layout": [_vp, _i32, _i32, _i32, _vp, _vp, _vp],
     "moe_ep_combine": [_vp, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _i32,
@@ -211,6 +213,17 @@ def moe_unpermute_combine(y, token_slot, topk_w, residual, out) -> None:
     _check("moe_unpermute_combine", _lib.moe_unpermute_combine(_p(y), _dt(y), _p(token_slot), _p(topk_w),
                                                                _p(residual), _dt(residual), T, d, k, _p(out),
                                                                _dt(out), _stream(residual.device)))
+
+
+def moe_grouped_swiglu_sized(xp, W_gate, W_up, W_down, counts, offsets, h, y, S_expected: int,
+                             dev_status=None) -> None:
+    """moe_grouped_swiglu over buffers of S_cap = xp.shape[0] rows, tiles chosen for S_expected rows."""
+    S, d = xp.shape
+    E, d_ff, _ = W_gate.shape
+    _check("moe_grouped_swiglu_sized",
+           _lib.moe_grouped_swiglu_sized(_p(xp), _p(W_gate), _p(W_up), _p(W_down), _dt(W_gate), _p(counts),
+                                         _p(offsets), S, S_expected, E, d, d_ff, _p(h), _p(y), _p(dev_status),
+                                         _stream(xp.device)))
 
 
 # --------------------------------------------------------------------------- expert parallelism over peer memory

@@ -232,6 +232,35 @@ moe_status_t moe_grouped_swiglu(const void* xp, const void* W_gate, const void* 
     return moe_expert_down(h, W_down, dt, counts, offsets, S, E, d, d_ff, y, dev_status, stream);
 }
 
+moe_status_t moe_grouped_swiglu_sized(const void* xp, const void* W_gate, const void* W_up, const void* W_down,
+                                      moe_dtype_t dt, const int32_t* counts, const int32_t* offsets, int32_t S_cap,
+                                      int32_t S_expected, int32_t E, int32_t d, int32_t d_ff, void* h, void* y,
+                                      int32_t* dev_status, moe_stream_t stream) {
+    moe_status_t st = check_expert_shape(dt, S_cap, E, d, d_ff);
+    if (st != MOE_OK) return st;
+    if (S_expected <= 0 || S_expected > S_cap) return MOE_ERR_INVALID_ARG;
+    if (!xp || !W_gate || !W_up || !W_down || !counts || !offsets || !h || !y) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(xp) || !aligned16(W_gate) || !aligned16(W_up) || !aligned16(W_down) || !aligned16(h) ||
+        !aligned16(y))
+        return MOE_ERR_INVALID_ARG;
+    Ctx c;
+    st = make_ctx(stream, c);
+    if (st != MOE_OK) return st;
+    if (dt == MOE_BF16) {
+        st = cuda_status(launch_gate_up_bf16(c, xp, W_gate, W_up, counts, offsets, S_cap, E, d, d_ff, h, dev_status,
+                                             nullptr, 0, 0, S_expected));
+        if (st != MOE_OK) return st;
+        return cuda_status(
+            launch_down_bf16(c, h, W_down, counts, offsets, S_cap, E, d, d_ff, y, dev_status, 0, S_expected));
+    }
+    st = cuda_status(launch_gate_up_f32(c, static_cast<const float*>(xp), static_cast<const float*>(W_gate),
+                                        static_cast<const float*>(W_up), counts, offsets, S_cap, E, d, d_ff,
+                                        static_cast<float*>(h)));
+    if (st != MOE_OK) return st;
+    return cuda_status(launch_down_f32(c, static_cast<const float*>(h), static_cast<const float*>(W_down), counts,
+                                       offsets, S_cap, E, d, d_ff, static_cast<float*>(y)));
+}
+
 moe_status_t moe_grouped_swiglu_masked(const void* x, const void* W_gate, const void* W_up, const void* W_down,
                                        moe_dtype_t dt, const int32_t* counts, int32_t E, int32_t cap, int32_t d,
                                        int32_t d_ff, void* h, void* y, int32_t* dev_status, moe_stream_t stream) {

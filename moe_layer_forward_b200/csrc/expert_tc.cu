@@ -563,15 +563,16 @@ bool gate_up_needs_permuted_rows(int S, int E) { return use_pair_gemm(S, E, 256)
 
 cudaError_t launch_gate_up_bf16(const Ctx& c, const void* xp, const void* Wg, const void* Wu, const int32_t* counts,
                                 const int32_t* offsets, int S, int E, int d, int d_ff, void* h, int32_t* status,
-                                const int32_t* gather, int act_rows, int cap) {
+                                const int32_t* gather, int act_rows, int cap, int S_sel) {
     if (S == 0) return cudaSuccess;
-    if (gather && (cap > 0 || gate_up_needs_permuted_rows(S, E))) return cudaErrorInvalidValue;
-    if (cap == 0 && use_pair_gemm(S, E, 256))
+    const int Ss = S_sel > 0 ? S_sel : S;  // rows the tile form is chosen for
+    if (gather && (cap > 0 || gate_up_needs_permuted_rows(Ss, E))) return cudaErrorInvalidValue;
+    if (cap == 0 && use_pair_gemm(Ss, E, 256))
         return launch_gate_up_bf16_pair(c, xp, Wg, Wu, counts, offsets, S, E, d, d_ff, h, status);
     tc::Args a{counts, offsets, E, d, d_ff, static_cast<uint16_t*>(h), (int64_t)d_ff, status, gather,
                static_cast<const uint16_t*>(xp), cap};
     const int ar = gather ? act_rows : -1;
-    switch (tc::pick_swap_rows(S, E)) {
+    switch (tc::pick_swap_rows(Ss, E)) {
         case 16: return tc::run<true, true, 16, 128>(c, xp, S, Wg, Wu, a, ar);
         case 32: return tc::run<true, true, 32, 128>(c, xp, S, Wg, Wu, a, ar);
         case 64: return tc::run<true, true, 64, 128>(c, xp, S, Wg, Wu, a, ar);
@@ -581,12 +582,13 @@ cudaError_t launch_gate_up_bf16(const Ctx& c, const void* xp, const void* Wg, co
 }
 
 cudaError_t launch_down_bf16(const Ctx& c, const void* h, const void* Wd, const int32_t* counts, const int32_t* offsets,
-                             int S, int E, int d, int d_ff, void* y, int32_t* status, int cap) {
+                             int S, int E, int d, int d_ff, void* y, int32_t* status, int cap, int S_sel) {
     if (S == 0) return cudaSuccess;
-    if (cap == 0 && use_pair_gemm(S, E, d))
+    const int Ss = S_sel > 0 ? S_sel : S;
+    if (cap == 0 && use_pair_gemm(Ss, E, d))
         return launch_down_bf16_pair(c, h, Wd, counts, offsets, S, E, d, d_ff, y, status);
     tc::Args a{counts, offsets, E, d_ff, d, static_cast<uint16_t*>(y), (int64_t)d, status, nullptr, nullptr, cap};
-    const int ra = tc::pick_rows(S, E);
+    const int ra = tc::pick_rows(Ss, E);
     if (d % 256 == 0) {
         switch (ra) {
             case 16: return tc::run<false, false, 16, 256>(c, h, S, Wd, nullptr, a);

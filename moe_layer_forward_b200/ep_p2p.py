@@ -23,9 +23,11 @@ source.  Here the travel is done by the kernels themselves:
 
 Rank r of N owns experts [r E/N, (r+1) E/N).  The buffers are sized for the
 worst case, N * T_max * min(k, E/N) rows (a token's k picks are distinct
-experts, at most E/N of them on one rank), so no count has to reach the host
-before the dispatch; the host reads the table once (overlapping the dispatch)
-to size the expert MLP call.
+experts, at most E/N of them on one rank), and the expert MLP runs over the
+whole buffer with its counts on the device (``moe_grouped_swiglu_sized``, tile
+form chosen for the rank's own slot count, which is what a rank receives on
+average), so no count ever reaches the host: the step has no host
+synchronisation and can be captured in a CUDA graph.
 
 ``ops`` and ``peers`` are parameters: on GPUs the library's kernels and
 peer-mapped buffers (``symmetric_peers`` over NVLink, or ``local_peers`` when
@@ -125,11 +127,13 @@ class CudaP2POps(CudaOps):
         self.m.moe_ep_layout(table, rank, counts_loc, offsets_loc)
         return counts_loc, offsets_loc
 
-    def expert_mlp(self, xp, W_gate, W_up, W_down, counts, offsets, y):
+    def expert_mlp(self, xp, W_gate, W_up, W_down, counts, offsets, y, S_expected):
+        """The grouped MLP over a whole receive buffer; counts/offsets on the device pick the rows."""
         S = xp.shape[0]
         if S > 0:
             h = torch.empty((S, W_gate.shape[1]), dtype=xp.dtype, device=xp.device)
-            self.m.moe_grouped_swiglu(xp, W_gate, W_up, W_down, counts, offsets, h, y)
+            self.m.moe_grouped_swiglu_sized(xp, W_gate, W_up, W_down, counts, offsets, h, y,
+                                            max(1, min(S_expected, S)))
 
     def combine_pull(self, peers: Peers, idx, token_slot, offsets, table, rank, w, residual, out_dtype):
         out = torch.empty(residual.shape, dtype=out_dtype, device=residual.device)
@@ -157,10 +161,6 @@ def _route(ops, x, gamma, W_r, b, E, top_k, eps, dtype) -> _Route:
     return _Route(idx, w, vx, counts, offsets, token_slot)
 
 
-def _received_rows(table_host: torch.Tensor, rank: int, E_loc: int) -> int:
-    return int(table_host[:, rank * E_loc:(rank + 1) * E_loc].sum())
-
-
 def _barrier(group, device):
     # a one-element all-reduce: ordered on the stream after this rank's preceding kernels, complete on every
     # rank only once all ranks reached it (no host wait on GPUs)
@@ -172,7 +172,8 @@ def ep_p2p_forward(x, gamma, W_r, b, W_gate_local, W_up_local, W_down_local, E: 
     """out = x + MoE(RMSNorm(x)) for this rank's tokens (one process per rank; collectives inside).
 
     W_*_local hold experts [rank E/N, (rank+1) E/N); peers holds buffers of at least
-    capacity_rows(T_max, N, top_k, E) rows on every rank.  Returns (out, EPStats)."""
+    capacity_rows(T_max, N, top_k, E) rows on every rank.  Returns (out, EPStats); the stats' rows_received
+    is a one-element device tensor (reading it is the only host synchronisation)."""
     ops = ops or CudaP2POps()
     N = dist.get_world_size(group)
     rank = dist.get_rank(group)
@@ -190,22 +191,16 @@ def ep_p2p_forward(x, gamma, W_r, b, W_gate_local, W_up_local, W_down_local, E: 
 
     table = torch.empty((N, E), dtype=torch.int32, device=dev)
     dist.all_gather(list(table.unbind(0)), rt.counts, group=group)
-    table_host = table.to("cpu", non_blocking=True)
-    done = torch.cuda.Event() if dev.type == "cuda" else None
-    if done is not None:
-        done.record()
     ops.dispatch(rt.vx, rt.idx, rt.token_slot, rt.offsets, table, rank, peers)
     _barrier(group, dev)
 
     counts_loc, offsets_loc = ops.layout(table, rank)
-    if done is not None:
-        done.synchronize()
-    R = _received_rows(table_host, rank, E_loc)
-    ops.expert_mlp(peers.recv[:R], W_gate_local, W_up_local, W_down_local, counts_loc, offsets_loc, peers.y[:R])
+    ops.expert_mlp(peers.recv, W_gate_local, W_up_local, W_down_local, counts_loc, offsets_loc, peers.y,
+                   int(x.shape[0]) * top_k)
     _barrier(group, dev)
 
     out = ops.combine_pull(peers, rt.idx, rt.token_slot, rt.offsets, table, rank, rt.w, x, out_dtype or x.dtype)
-    return out, EPStats(rows_sent=int(x.shape[0]) * top_k, rows_received=R)
+    return out, EPStats(rows_sent=int(x.shape[0]) * top_k, rows_received=offsets_loc[E_loc:])
 
 
 def ep_p2p_forward_emulated(x_shards, gamma, W_r, b, W_gate, W_up, W_down, top_k: int = 8, eps: float = 1e-5,
@@ -228,12 +223,10 @@ def ep_p2p_forward_emulated(x_shards, gamma, W_r, b, W_gate, W_up, W_down, top_k
     table = torch.stack([rt.counts for rt in routes])  # what the all-gather gives every rank
     for r, rt in enumerate(routes):
         ops.dispatch(rt.vx, rt.idx, rt.token_slot, rt.offsets, table, r, peers[r])
-    table_host = table.cpu()
     for j in range(N):
         counts_loc, offsets_loc = ops.layout(table, j)
-        R = _received_rows(table_host, j, E_loc)
         sl = slice(j * E_loc, (j + 1) * E_loc)
-        ops.expert_mlp(peers[j].recv[:R], W_gate[sl], W_up[sl], W_down[sl], counts_loc, offsets_loc,
-                       peers[j].y[:R])
+        ops.expert_mlp(peers[j].recv, W_gate[sl], W_up[sl], W_down[sl], counts_loc, offsets_loc, peers[j].y,
+                       int(x_shards[j].shape[0]) * top_k)
     return [ops.combine_pull(peers[r], rt.idx, rt.token_slot, rt.offsets, table, r, rt.w, x_shards[r],
                              out_dtype or x_shards[r].dtype) for r, rt in enumerate(routes)]

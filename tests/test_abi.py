@@ -159,6 +159,35 @@ def test_expert_and_combine_reject_bad_shapes_on_host(lib):
     assert c(_p(), 1, _p(), _p(), _p(), 5, 4, 64, 8, _p(), 1, NULL) == INVALID
 
 
+def test_peer_memory_and_sized_entries_reject_bad_arguments_on_host(lib):
+    i32 = ctypes.c_int32
+    sz = lib.moe_grouped_swiglu_sized
+    sz.argtypes = [V, V, V, V, ctypes.c_int, V, V, i32, i32, i32, i32, i32, V, V, V, V]
+    assert sz(_p(), _p(), _p(), _p(), 1, _p(), _p(), 64, 0, 8, 128, 256, _p(), _p(), NULL, NULL) == INVALID
+    assert sz(_p(), _p(), _p(), _p(), 1, _p(), _p(), 64, 65, 8, 128, 256, _p(), _p(), NULL, NULL) == INVALID
+    assert sz(_p(), _p(), _p(), _p(), 1, _p(), _p(), 64, 32, 8, 96, 256, _p(), _p(), NULL, NULL) == UNSUPPORTED
+    assert sz(_p(), _p(), _p(), _p(), 1, NULL, _p(), 64, 32, 8, 128, 256, _p(), _p(), NULL, NULL) == INVALID
+    dsp = lib.moe_ep_dispatch
+    dsp.argtypes = [V, ctypes.c_int, V, V, V, V, i32, i32, i32, i32, i32, i32, V, V, V]
+    assert dsp(_p(), 1, _p(), _p(), _p(), _p(), 0, 3, 16, 4, 64, 8, _p(), NULL, NULL) == UNSUPPORTED  # E % N
+    assert dsp(_p(), 1, _p(), _p(), _p(), _p(), 2, 2, 16, 4, 64, 8, _p(), NULL, NULL) == INVALID  # rank < N
+    assert dsp(_p(), 1, _p(), _p(), _p(), NULL, 0, 2, 16, 4, 64, 8, _p(), NULL, NULL) == INVALID  # table
+    assert dsp(_p(), 1, _p(), _p(), _p(), _p(), 0, 2, 16, 4, 60, 8, _p(), NULL, NULL) == UNSUPPORTED  # d % 8
+    assert dsp(_p(), 1, _p(), _p(), _p(), _p(), 0, 2, 16, 4, 64, 8, NULL, NULL, NULL) == INVALID  # recv_bufs
+    assert dsp(_p(), 1, _p(), _p(), _p(), _p(), 0, 2, 16, 0, 64, 8, _p(), NULL, NULL) == OK  # no tokens
+    lay = lib.moe_ep_layout
+    lay.argtypes = [V, i32, i32, i32, V, V, V]
+    assert lay(NULL, 0, 2, 16, _p(), _p(), NULL) == INVALID
+    assert lay(_p(), 0, 2, 16, NULL, _p(), NULL) == INVALID
+    assert lay(_p(), 0, 5, 16, _p(), _p(), NULL) == UNSUPPORTED
+    cmb = lib.moe_ep_combine
+    cmb.argtypes = [V, ctypes.c_int, V, V, V, V, i32, i32, i32, V, V, ctypes.c_int, i32, i32, i32, V, ctypes.c_int, V,
+                    V]
+    assert cmb(_p(), 1, _p(), _p(), _p(), _p(), 0, 2, 16, _p(), _p(), 1, 4, 64, 9, _p(), 1, NULL, NULL) == UNSUPPORTED
+    assert cmb(NULL, 1, _p(), _p(), _p(), _p(), 0, 2, 16, _p(), _p(), 1, 4, 64, 8, _p(), 1, NULL, NULL) == INVALID
+    assert cmb(_p(), 1, _p(), _p(), _p(), _p(), 0, 2, 16, _p(), _p(), 7, 4, 64, 8, _p(), 1, NULL, NULL) == INVALID
+
+
 class Shape(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("E", ctypes.c_int32), ("top_k", ctypes.c_int32),
                 ("d_ff", ctypes.c_int32), ("eps", ctypes.c_float), ("x_dtype", ctypes.c_int),

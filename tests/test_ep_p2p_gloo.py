@@ -70,9 +70,10 @@ def _p2p_ops():
             offsets[1:] = torch.cumsum(counts, 0)
             return counts, offsets
 
-        def expert_mlp(self, xp, W_gate, W_up, W_down, counts, offsets, y):
-            if xp.shape[0]:
-                y.copy_(self.grouped_swiglu(xp, W_gate, W_up, W_down, counts, offsets))
+        def expert_mlp(self, xp, W_gate, W_up, W_down, counts, offsets, y, S_expected):
+            R = int(offsets[-1])
+            if R:
+                y[:R].copy_(self.grouped_swiglu(xp[:R], W_gate, W_up, W_down, counts, offsets))
 
         def combine_pull(self, peers, idx, token_slot, offsets, table, rank, w, residual, out_dtype):
             E_loc = table.shape[1] // table.shape[0]
@@ -109,7 +110,7 @@ def _worker(rank, world, port, outdir, recv, y):
     out, stats = ep_p2p.ep_p2p_forward(x, I["gamma"], I["W_r"], I["b"], I["W_gate"][experts], I["W_up"][experts],
                                        I["W_down"][experts], E=w.E, peers=peers, T_max=T_max, top_k=w.top_k,
                                        eps=w.eps, ops=_p2p_ops())
-    torch.save({"out": out, "received": stats.rows_received}, os.path.join(outdir, f"r{rank}.pt"))
+    torch.save({"out": out, "received": int(stats.rows_received)}, os.path.join(outdir, f"r{rank}.pt"))
     dist.barrier()
     dist.destroy_process_group()
 

@@ -125,6 +125,31 @@ def test_ranks_exchange_exactly_and_match_the_oracle(moe, N, shape):
     assert max_abs <= MAX_ABS and rel <= REL_L2, (max_abs, rel)
 
 
+def test_sized_grouped_mlp_equals_the_exact_call(moe):
+    # a buffer of S_cap rows of which the counts use S: the same rows as moe_grouped_swiglu on exactly S rows,
+    # and the rows past the segments are left as they were
+    S, S_cap, d, d_ff = 200, 256, 256, 384
+    counts = torch.tensor([30, 0, 7, 41, 12, 1, 50, 59], dtype=torch.int32)
+    E = counts.numel()
+    offsets = torch.zeros(E + 1, dtype=torch.int32)
+    offsets[1:] = torch.cumsum(counts, 0)
+    assert int(offsets[-1]) == S
+    W = [synth.normal((E, n, kk), 970, 5 + i, 0.0, 1 / kk ** 0.5, torch.bfloat16).to(DEV)
+         for i, (n, kk) in enumerate([(d_ff, d), (d_ff, d), (d, d_ff)])]
+    xp = torch.full((S_cap, d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    xp[:S] = synth.normal((S, d), 970, 1, dtype=torch.bfloat16).to(DEV)
+    c, o = counts.to(DEV), offsets.to(DEV)
+    h_ref = torch.empty((S, d_ff), dtype=torch.bfloat16, device=DEV)
+    y_ref = torch.empty((S, d), dtype=torch.bfloat16, device=DEV)
+    moe.moe_grouped_swiglu(xp[:S].contiguous(), *W, c, o, h_ref, y_ref)
+    h = torch.empty((S_cap, d_ff), dtype=torch.bfloat16, device=DEV)
+    y = torch.full((S_cap, d), 7.0, dtype=torch.bfloat16, device=DEV)
+    moe.moe_grouped_swiglu_sized(xp, *W, c, o, h, y, S)
+    torch.cuda.synchronize()
+    assert torch.equal(y[:S], y_ref)
+    assert (y[S:] == 7.0).all()
+
+
 def _free_port() -> int:
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
@@ -152,7 +177,7 @@ def _driver_worker(rank, port, outdir, shape):
     m.moe_forward(D["x"], D["gamma"], D["W_r"], D["b"], D["W_gate"], D["W_up"], D["W_down"], ref, top_k=w.top_k,
                   eps=w.eps)
     torch.cuda.synchronize()
-    torch.save({"equal": torch.equal(out, ref), "rows": stats.rows_received}, os.path.join(outdir, "r.pt"))
+    torch.save({"equal": torch.equal(out, ref), "rows": int(stats.rows_received)}, os.path.join(outdir, "r.pt"))
     dist.destroy_process_group()
 
 
