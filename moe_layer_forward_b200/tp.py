@@ -14,7 +14,9 @@ holds all tokens.  One step:
   2. the grouped SwiGLU MLP on the rank's d_ff slice: a partial y;
   3. the weighted combine of the partial y in fp32, with the residual added on
      rank 0 only, then one fp32 all-reduce (sum) across the ranks, and a cast
-     to the output dtype.
+     to the output dtype.  With ``scatter=True`` the sum is a reduce-scatter
+     over tokens instead: rank r receives tokens [r T/N, (r+1) T/N) (T
+     divisible by N), the form that feeds a token-sharded next layer.
 
 All arithmetic runs in the library's kernels (``ops``, as in ``ep``); the
 reduction is ``torch.distributed.all_reduce`` (NCCL on GPUs).
@@ -28,10 +30,15 @@ from .ep import CudaOps
 
 
 def tp_forward(x, gamma, W_r, b, W_gate_slice, W_up_slice, W_down_slice, top_k: int = 8, eps: float = 1e-5,
-               group=None, ops=None, out_dtype=None):
-    """out = x + MoE(RMSNorm(x)) with this rank's d_ff slice of every expert (collective over ``group``)."""
+               group=None, ops=None, out_dtype=None, scatter: bool = False):
+    """out = x + MoE(RMSNorm(x)) with this rank's d_ff slice of every expert (collective over ``group``).
+
+    scatter=False: every rank returns all T rows; scatter=True: rank r returns rows [r T/N, (r+1) T/N)."""
     ops = ops or CudaOps()
     rank = dist.get_rank(group)
+    N = dist.get_world_size(group)
+    if scatter and x.shape[0] % N != 0:
+        raise ValueError(f"{x.shape[0]} tokens do not split over {N} ranks")
     E = W_gate_slice.shape[0]
     out_dtype = out_dtype or x.dtype
     if W_down_slice.shape[2] != W_gate_slice.shape[1]:
@@ -43,5 +50,9 @@ def tp_forward(x, gamma, W_r, b, W_gate_slice, W_up_slice, W_down_slice, top_k: 
     y_part = ops.grouped_swiglu(xp, W_gate_slice, W_up_slice, W_down_slice, counts, offsets)
     residual = x if rank == 0 else torch.zeros_like(x)
     part = ops.combine(y_part, token_slot, w, residual, torch.float32)
+    if scatter:
+        mine = torch.empty((x.shape[0] // N, part.shape[1]), dtype=part.dtype, device=part.device)
+        dist.reduce_scatter_tensor(mine, part, op=dist.ReduceOp.SUM, group=group)
+        return mine.to(out_dtype)
     dist.all_reduce(part, op=dist.ReduceOp.SUM, group=group)
     return part.to(out_dtype)

@@ -168,6 +168,48 @@ def test_tensor_parallel_layer_equals_the_single_process_layer(world):
     assert torch.allclose(r[0].double(), ref, rtol=1e-5, atol=1e-5)
 
 
+def _tp_scatter_worker(rank, world, port, outdir):
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import datetime
+
+    import torch.distributed as dist
+
+    from moe_layer_forward_b200 import tp
+
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    w, I = _tp_inputs()
+    F = w.d_ff // world
+    f = slice(rank * F, (rank + 1) * F)
+    out = tp.tp_forward(I["x"], I["gamma"], I["W_r"], I["b"], I["W_gate"][:, f].contiguous(),
+                        I["W_up"][:, f].contiguous(), I["W_down"][:, :, f].contiguous(), top_k=w.top_k, eps=w.eps,
+                        ops=OracleOps(), scatter=True)
+    torch.save({"out": out}, os.path.join(outdir, f"r{rank}.pt"))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_tensor_parallel_reduce_scatter_gives_each_rank_its_tokens(world):
+    sys.path.insert(0, ROOT)
+    w, I = _tp_inputs()
+    ops = OracleOps()
+    v32 = ops.rmsnorm(I["x"], I["gamma"], w.eps, torch.float32)
+    idx, wt = ops.router(v32, I["W_r"], I["b"], w.top_k)
+    counts, offsets, token_slot, xp = ops.permute(v32, idx, w.E)
+    y = ops.grouped_swiglu(xp, I["W_gate"], I["W_up"], I["W_down"], counts, offsets)
+    ref = ops.combine(y, token_slot, wt, I["x"], torch.float64)
+    with tempfile.TemporaryDirectory() as d:
+        mp.start_processes(_tp_scatter_worker, args=(world, _free_port(), d), nprocs=world, join=True,
+                           start_method="spawn")
+        r = [torch.load(os.path.join(d, f"r{k}.pt"))["out"] for k in range(world)]
+    T_r = w.T // world
+    for k in range(world):  # rank k holds tokens [k T/N, (k+1) T/N), the regrouped sum as in the all-reduce form
+        assert r[k].shape[0] == T_r
+        assert torch.allclose(r[k].double(), ref[k * T_r:(k + 1) * T_r], rtol=1e-5, atol=1e-5)
+
+
 def _single_rank_group(port):
     import datetime
 
