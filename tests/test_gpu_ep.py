@@ -48,9 +48,11 @@ def _worker(rank, port, outdir, shape):
 
     out_tp = tp.tp_forward(D["x"], D["gamma"], D["W_r"], D["b"], D["W_gate"], D["W_up"], D["W_down"], top_k=w.top_k,
                            eps=w.eps)
+    out_tps = tp.tp_forward(D["x"], D["gamma"], D["W_r"], D["b"], D["W_gate"], D["W_up"], D["W_down"],
+                            top_k=w.top_k, eps=w.eps, scatter=True)
     torch.cuda.synchronize()
-    torch.save({"equal": torch.equal(out_ep, out), "tp_equal": torch.equal(out_tp, out), "rows": stats.rows_received},
-               os.path.join(outdir, "r.pt"))
+    torch.save({"equal": torch.equal(out_ep, out), "tp_equal": torch.equal(out_tp, out) and torch.equal(out_tps, out),
+                "rows": stats.rows_received}, os.path.join(outdir, "r.pt"))
     dist.destroy_process_group()
 
 

@@ -11,7 +11,8 @@ another).  Checks:
     every rank's output equals moe_unpermute_combine over the expert rows
     gathered by that layout, bit for bit; the layer is within the parity
     tolerances of the fp64 oracle on the GPU's routing;
-  - the per-rank driver (NCCL group of one, spawned) equals moe_forward.
+  - the per-rank driver (NCCL group of one, spawned) equals moe_forward;
+  - two emulated ranks replay from a CUDA graph (no host synchronisation).
 """
 import os
 import socket
@@ -123,6 +124,38 @@ def test_ranks_exchange_exactly_and_match_the_oracle(moe, N, shape):
     forced = oracle.moe_layer(I["x"], *args, k=w.top_k, eps=w.eps, force_idx=idx, force_w=wt)
     max_abs, rel = errors(torch.cat([o.cpu() for o in outs]), forced["out"])
     assert max_abs <= MAX_ABS and rel <= REL_L2, (max_abs, rel)
+
+
+def test_two_ranks_replay_from_a_cuda_graph(moe):
+    # the step has no host synchronisation: captured once, a replay reproduces the eager result, also after a
+    # replay on other inputs
+    from moe_layer_forward_b200 import ep_p2p
+
+    w, I, D = _inputs((96, 512, 64, 256), 980)
+    N = 2
+    shards = [s.contiguous() for s in D["x"].chunk(N)]  # views of D["x"]
+    peers = ep_p2p.local_peers(N, ep_p2p.capacity_rows(48, N, 8, 64), 512, torch.bfloat16, DEV)
+    args = (D["gamma"], D["W_r"], D["b"], D["W_gate"], D["W_up"], D["W_down"])
+    eager = [o.clone() for o in ep_p2p.ep_p2p_forward_emulated(shards, *args, peers=peers)]
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        ep_p2p.ep_p2p_forward_emulated(shards, *args, peers=peers)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        outs = ep_p2p.ep_p2p_forward_emulated(shards, *args, peers=peers)
+    saved = [x.clone() for x in shards]
+    for x in shards:
+        x.zero_()
+    g.replay()
+    for x, src in zip(shards, saved):
+        x.copy_(src)
+    g.replay()
+    torch.cuda.synchronize()
+    assert all(torch.equal(a, b) for a, b in zip(outs, eager))
+    del g
 
 
 def test_sized_grouped_mlp_equals_the_exact_call(moe):
