@@ -173,7 +173,9 @@ def ep_p2p_forward(x, gamma, W_r, b, W_gate_local, W_up_local, W_down_local, E: 
 
     W_*_local hold experts [rank E/N, (rank+1) E/N); peers holds buffers of at least
     capacity_rows(T_max, N, top_k, E) rows on every rank.  Returns (out, EPStats); the stats' rows_received
-    is a one-element device tensor (reading it is the only host synchronisation)."""
+    is a one-element device tensor (reading it is the only host synchronisation).  The argument checks run
+    before the first collective: a rank that fails one raises at once, and the other ranks' next collective
+    ends with the process group's timeout error."""
     ops = ops or CudaP2POps()
     N = dist.get_world_size(group)
     rank = dist.get_rank(group)
