@@ -151,3 +151,47 @@ def test_capacity_covers_the_worst_case():
     # every token of every rank sends min(k, E/N) rows to one rank at most
     assert ep_p2p.capacity_rows(10, 4, 8, 16) == 4 * 10 * 4
     assert ep_p2p.capacity_rows(10, 2, 8, 64) == 2 * 10 * 8
+
+
+def _failing_worker(rank, world, port, outdir, recv, y):
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import datetime
+
+    import torch.distributed as dist
+
+    from moe_layer_forward_b200 import ep_p2p
+
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=5))
+    w, I = _inputs()
+    E_loc = w.E // world
+    experts = slice(rank * E_loc, (rank + 1) * E_loc)
+    x = I["x"].chunk(world)[rank].contiguous()
+    T_max = x.shape[0] - (1 if rank == 1 else 0)  # rank 1 holds one token more than the buffers were sized for
+    outcome = "returned"
+    try:
+        ep_p2p.ep_p2p_forward(x, I["gamma"], I["W_r"], I["b"], I["W_gate"][experts], I["W_up"][experts],
+                              I["W_down"][experts], E=w.E, peers=ep_p2p.Peers(recv[rank], y[rank], recv, y),
+                              T_max=T_max, top_k=w.top_k, eps=w.eps, ops=_p2p_ops())
+    except ValueError as e:
+        outcome = "ValueError: " + str(e)
+    except RuntimeError as e:  # the collective that the failed rank never joins
+        outcome = "RuntimeError"
+    torch.save({"outcome": outcome}, os.path.join(outdir, f"r{rank}.pt"))
+
+
+def test_a_rank_that_fails_its_checks_ends_the_others_collective_with_an_error():
+    from moe_layer_forward_b200 import ep_p2p
+
+    world = 2
+    w, I = _inputs()
+    rows = ep_p2p.capacity_rows(w.T // world, world, w.top_k, w.E)
+    recv = [torch.zeros((rows, w.d), dtype=torch.float32).share_memory_() for _ in range(world)]
+    y = [torch.zeros((rows, w.d), dtype=torch.float64).share_memory_() for _ in range(world)]
+    with tempfile.TemporaryDirectory() as d:
+        mp.start_processes(_failing_worker, args=(world, _free_port(), d, recv, y), nprocs=world, join=True,
+                           start_method="spawn")
+        r = [torch.load(os.path.join(d, f"r{k}.pt"))["outcome"] for k in range(world)]
+    assert r[1].startswith("ValueError") and "T_max" in r[1]
+    assert r[0] == "RuntimeError"
