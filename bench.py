@@ -5,7 +5,12 @@
 
 One step = one whole layer forward R = X + MoE(RMSNorm(X)) (RMSNorm, router,
 permutation, grouped SwiGLU expert MLP, combine) over one batch of seeded
-synthetic tokens, inputs resident in HBM.  Prints one JSON line (rank 0).
+synthetic tokens, inputs resident in HBM.  Prints one JSON line (rank 0): the
+headline workload (decode by default) at the top level and, at one GPU, all
+five workloads (tiny, decode, prefill, skewed, block) under "workloads", each
+with tokens/s, the layer's fraction of its roofline, the dominant kernel's
+fraction, the near-tie token count, end-to-end throughput and a CPU oracle
+sample.
 
 With N > 1 (torchrun) every rank runs an independent replica on its own GPU
 (tokens are independent; there is no data-path collective) and the time is
@@ -40,7 +45,10 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="decode", help="tiny | decode | prefill | skewed | block")
+    ap.add_argument("--workload", default="decode", help="headline workload: tiny | decode | prefill | skewed | block")
+    ap.add_argument("--workloads", choices=["all", "one"], default="all",
+                    help="all: at one GPU, also measure the other four workloads (reported under 'workloads'); "
+                         "one: the headline workload only")
     ap.add_argument("--shrink", type=int, default=1,
                     help="divide T and E by this factor (same rows per expert, smaller device footprint); "
                          "for ncu captures of the same kernels, never for reported numbers")
@@ -85,8 +93,9 @@ def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         j = json.load(open(p))
-        return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"], "source": "measured"}
-    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+        return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"],
+                "bf16_tflops_sustained": j.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
 class Clocks:
@@ -168,10 +177,10 @@ def oracle_tokens_per_s(I, w, n_tokens: int, start: int = 0):
     return n_tokens / dt, dt
 
 
-def cpu_baseline(I, w):
-    # one token first to size a sample of about 15 s of single-core work
+def cpu_baseline(I, w, seconds: float = 15.0):
+    # one token first to size a sample of about `seconds` of single-core work
     _, t1 = oracle_tokens_per_s(I, w, 1)
-    n = int(max(1, min(256, 15.0 / max(t1, 1e-3))))
+    n = int(max(1, min(256, seconds / max(t1, 1e-3))))
     v, dt = oracle_tokens_per_s(I, w, n, start=1)
     return {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
             "sample": f"{n} token rows cycling through the {w.T} of the {w.name} workload, whole layer per "
@@ -205,72 +214,136 @@ def run_reference(a, w):
     return 0
 
 
+def active_weight_bytes(w) -> int:
+    esz = 2 if str(w.w_dtype).endswith("bfloat16") else 4
+    return w.E * 3 * w.d * w.d_ff * esz
+
+
 def config_of(w, n):
     return {"workload": w.name, "T": w.T, "d": w.d, "E": w.E, "top_k": w.top_k, "d_ff": w.d_ff,
             "x_dtype": str(w.x_dtype).replace("torch.", ""), "expert_dtype": str(w.w_dtype).replace("torch.", ""),
             "out_dtype": str(w.out_dtype).replace("torch.", ""), "global_batch_tokens": w.T * n,
             "parallelism": "replicas" if n > 1 else "single",
-            "l2": "not flushed: every step streams the active experts' weights, many times the 126 MB L2"}
+            "l2": "not flushed: inputs larger than L2 (every step streams the active experts' weights, "
+                  f"{active_weight_bytes(w) / 1e9:.1f} GB at most, against the 126 MB L2)"}
 
 
 # --------------------------------------------------------------------------- GPU arm
-def run_ours(a, w):
+def _timed(fn, steps: int, warmup: int, barrier, clocks_gpu=None):
+    """(device ms over exactly `steps` calls of fn, clock summary or None, launches): CUDA events on the
+    current stream, a barrier and a device synchronisation on both sides, after `warmup` untimed calls."""
     import torch
-    import torch.distributed as dist
 
     import moe_layer_forward_b200 as moe
-    import synth
 
-    rank, world, local = dist_env()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
-
-    I = synth.make_layer_inputs(w)
-    D = {n: t.to(dev) for n, t in I.items()}
-    T, k, E = w.T, w.top_k, w.E
-    out = torch.empty((T, w.d), dtype=w.out_dtype, device=dev)
-    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
-    wt = torch.empty((T, k), dtype=torch.float32, device=dev)
-    status = torch.zeros(1, dtype=torch.int32, device=dev)
-    ws = torch.empty(moe.forward_workspace_bytes(D["x"], D["W_r"], D["W_gate"], out, k, w.eps), dtype=torch.uint8,
-                     device=dev)
-
-    def step(x=None, o=None):
-        moe.moe_forward(D["x"] if x is None else x, D["gamma"], D["W_r"], D["b"], D["W_gate"], D["W_up"],
-                        D["W_down"], out if o is None else o, top_k=k, eps=w.eps, topk_idx=idx, topk_w=wt, ws=ws,
-                        dev_status=status)
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-
-    max_over_ranks = reduce_max_fn(dist, dev)
-
-    for _ in range(a.warmup):
-        step()
-    torch.cuda.synchronize()
-    if status.item() != 0:
-        raise RuntimeError(f"device status {status.item()} after warm-up")
-
-    # ---- timed region: exactly K steps, device-resident inputs
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(warmup):
+        fn()
     barrier()
-    with Clocks(local) as clk:
-        n0 = moe.kernel_launches()
-        e0.record()
-        for _ in range(a.steps):
-            step()
-        e1.record()
-        launches = moe.kernel_launches() - n0  # counted by the library itself
-        barrier()
-    value, ms_per_step = aggregate(e0.elapsed_time(e1), T, a.steps, world, max_over_ranks)
-    if status.item() != 0:
-        raise RuntimeError(f"device status {status.item()} in the timed region")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clk = Clocks(clocks_gpu) if clocks_gpu is not None else None
+    if clk:
+        clk.__enter__()
+    n0 = moe.kernel_launches()
+    e0.record()
+    for _ in range(steps):
+        fn()
+    e1.record()
+    launches = moe.kernel_launches() - n0
+    barrier()
+    if clk:
+        clk.__exit__(None, None, None)
+    return e0.elapsed_time(e1), (clk.summary() if clk else None), launches
 
-    # ---- dominant kernel (expert gate/up GEMM) timed per launch through the step-level entry points
+
+def layer_roofline(w, active: int, ms: float, pk: dict) -> dict:
+    """The whole layer against its binding roofline: algorithmic bytes (active experts' weights, X, R, W_r,
+    gamma, b) over the measured copy peak, or expert-GEMM flops (6 S d d_ff) over the measured bf16 peak."""
+    esz = 2 if str(w.w_dtype).endswith("bfloat16") else 4
+    xsz = 2 if str(w.x_dtype).endswith("bfloat16") else 4
+    osz = 2 if str(w.out_dtype).endswith("bfloat16") else 4
+    nbytes = active * 3 * w.d * w.d_ff * esz + w.T * w.d * (xsz + osz) + w.E * w.d * 4 + w.d * 4 + w.E * 4
+    flops = 6.0 * w.T * w.top_k * w.d * w.d_ff
+    t = ms / 1000.0
+    t_hbm = nbytes / (pk["hbm_gbs"] * 1e9)
+    t_tc = flops / (pk["bf16_tflops"] * 1e12)
+    r = {"algorithmic_bytes": nbytes, "expert_flops": flops,
+         "hbm_gbs": nbytes / t / 1e9, "hbm_frac": nbytes / t / 1e9 / pk["hbm_gbs"],
+         "tensor_tflops": flops / t / 1e12, "tensor_frac": flops / t / 1e12 / pk["bf16_tflops"],
+         "t_roof_ms": 1000.0 * max(t_hbm, t_tc)}
+    if t_hbm >= t_tc:
+        r.update(bound="hbm", frac=r["hbm_frac"], peak=pk["hbm_gbs"], unit="GB/s", achieved=r["hbm_gbs"])
+    else:
+        r.update(bound="tensor", frac=r["tensor_frac"], peak=pk["bf16_tflops"], unit="TFLOP/s",
+                 achieved=r["tensor_tflops"])
+        if pk.get("bf16_tflops_sustained"):
+            r["frac_sustained"] = r["tensor_tflops"] / pk["bf16_tflops_sustained"]
+    r["peak_source"] = pk["source"]
+    return r
+
+
+class Layer:
+    """One workload's inputs, outputs and workspace on the device, and its step through moe_forward."""
+
+    def __init__(self, w, dev):
+        import torch
+
+        import moe_layer_forward_b200 as moe
+        import synth
+
+        self.w, self.dev = w, dev
+        self.I = synth.make_layer_inputs(w)
+        self.D = {n: t.to(dev) for n, t in self.I.items()}
+        T, k, E = w.T, w.top_k, w.E
+        self.out = torch.empty((T, w.d), dtype=w.out_dtype, device=dev)
+        self.idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+        self.wt = torch.empty((T, k), dtype=torch.float32, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.ws = torch.empty(moe.forward_workspace_bytes(self.D["x"], self.D["W_r"], self.D["W_gate"], self.out, k,
+                                                          w.eps), dtype=torch.uint8, device=dev)
+
+    def step(self, x=None):
+        import moe_layer_forward_b200 as moe
+
+        D, w = self.D, self.w
+        moe.moe_forward(D["x"] if x is None else x, D["gamma"], D["W_r"], D["b"], D["W_gate"], D["W_up"],
+                        D["W_down"], self.out, top_k=w.top_k, eps=w.eps, topk_idx=self.idx, topk_w=self.wt,
+                        ws=self.ws, dev_status=self.status)
+
+    def check_status(self, where: str):
+        if self.status.item() != 0:
+            raise RuntimeError(f"{self.w.name}: device status {self.status.item()} {where}")
+
+
+def near_ties(L) -> dict:
+    """Tokens whose 8th-to-9th selection-score margin is below 1e-5, from the library's own router (fp32
+    normalised rows, as moe_forward routes them); a diagnostic, outside every timed region."""
+    import torch
+
+    import moe_layer_forward_b200 as moe
+
+    w, D, dev = L.w, L.D, L.dev
+    if w.E <= w.top_k:
+        return {"count": 0, "threshold": 1e-5, "tokens": w.T}
+    v32 = torch.empty((w.T, w.d), dtype=torch.float32, device=dev)
+    moe.moe_rmsnorm(D["x"], D["gamma"], w.eps, v32)
+    idx = torch.empty((w.T, w.top_k), dtype=torch.int32, device=dev)
+    wt = torch.empty((w.T, w.top_k), dtype=torch.float32, device=dev)
+    margin = torch.empty(w.T, dtype=torch.float32, device=dev)
+    moe.moe_router_topk(v32, D["W_r"], D["b"], idx, wt, margin=margin)
+    n = int((margin < 1e-5).sum().item())
+    return {"count": n, "threshold": 1e-5, "tokens": w.T,
+            "same_routing_as_forward": bool(torch.equal(idx, L.idx))}
+
+
+def staged(L, a, barrier, pk) -> tuple:
+    """Per-step CUDA-event times of the six step-level entry points (a permuted copy feeds the GEMMs), and the
+    dominant kernel's (the gate/up GEMM's) roofline object."""
+    import torch
+
+    import moe_layer_forward_b200 as moe
+
+    w, D, dev = L.w, L.D, L.dev
+    T, k, E = w.T, w.top_k, w.E
     counts = torch.empty(E, dtype=torch.int32, device=dev)
     offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
     slot_token = torch.empty(T * k, dtype=torch.int32, device=dev)
@@ -279,10 +352,11 @@ def run_ours(a, w):
     xp = torch.empty((T * k, w.d), dtype=w.w_dtype, device=dev)
     h = torch.empty((T * k, w.d_ff), dtype=w.w_dtype, device=dev)
     y = torch.empty((T * k, w.d), dtype=w.w_dtype, device=dev)
+    idx, wt, out = torch.empty_like(L.idx), torch.empty_like(L.wt), torch.empty_like(L.out)
     names = ["rmsnorm", "router", "permute", "gate_up", "down", "combine"]
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(a.steps)]
 
-    def staged(ev=None):
+    def run(ev=None):
         rec = (lambda i: ev[i].record()) if ev else (lambda i: None)
         rec(0)
         moe.moe_rmsnorm(D["x"], D["gamma"], w.eps, v)
@@ -299,10 +373,10 @@ def run_ours(a, w):
         rec(6)
 
     for _ in range(a.warmup):
-        staged()
+        run()
     barrier()
     for i in range(a.steps):
-        staged(evs[i])
+        run(evs[i])
     torch.cuda.synchronize()
     stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(a.steps))
                 for j, n in enumerate(names)}
@@ -311,7 +385,6 @@ def run_ours(a, w):
     esz = 2 if w.w_dtype == torch.bfloat16 else 4
     gate_up_bytes = active * 2 * w.d_ff * w.d * esz + S * w.d * esz + S * w.d_ff * esz
     gate_up_flops = 2.0 * S * w.d * 2 * w.d_ff
-    pk = peaks()
     t_s = stage_ms["gate_up"] / 1000.0
     hbm_bound = gate_up_bytes / (pk["hbm_gbs"] * 1e9) >= gate_up_flops / (pk["bf16_tflops"] * 1e12)
     if hbm_bound:
@@ -326,9 +399,44 @@ def run_ours(a, w):
     roof["algorithmic_flops_per_launch"] = gate_up_flops
     roof["launch_ms"] = stage_ms["gate_up"]
     roof["peak_source"] = f"{pk['source']} (burst, kernel timed alone)"
+    return stage_ms, roof, active, (counts, offsets, xp)
 
-    # ---- the expert MLP on the masked layout ([E][cap][d] buffers + counts), same routing
-    masked = None
+
+def e2e_of(L, a, barrier, world, max_over_ranks) -> dict:
+    """The same layer through moe_forward with the step's input copied from pinned host memory and its
+    output read back to the host every step, inside the timed region."""
+    import torch
+
+    x_host = L.I["x"].pin_memory()
+    out_host = torch.empty(L.out.shape, dtype=L.out.dtype).pin_memory()
+    x_dev = torch.empty_like(L.D["x"])
+
+    def one():
+        x_dev.copy_(x_host, non_blocking=True)
+        L.step(x_dev)
+        out_host.copy_(L.out, non_blocking=True)
+        torch.cuda.current_stream().synchronize()  # the host reads this step's result
+
+    ms, _, _ = _timed(one, a.steps, a.warmup, barrier)
+    value, _ = aggregate(ms, L.w.T, a.steps, world, max_over_ranks)
+    return {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
+            "d2h_bytes_per_step": out_host.numel() * out_host.element_size()}
+
+
+def headline_extras(L, a, barrier, pk, ms_per_step, staged_bufs, active) -> dict:
+    """Next-row measurements on the headline workload: the masked layout, block-FP8 experts, and one rank of
+    the peer-memory expert-parallel step."""
+    import torch
+
+    import moe_layer_forward_b200 as moe
+
+    w, D, dev, status = L.w, L.D, L.dev, L.status
+    T, k, E = w.T, w.top_k, w.E
+    S = T * k
+    esz = 2 if w.w_dtype == torch.bfloat16 else 4
+    counts, offsets, xp = staged_bufs
+    res = {"masked_layout": None, "fp8_layer": None, "ep_p2p": None}
+
     if not a.no_masked and w.w_dtype == torch.bfloat16 and S // E <= 32:
         cn, of = counts.cpu(), offsets.cpu()
         cap = int((int(cn.max()) + 15) // 16 * 16)
@@ -337,126 +445,126 @@ def run_ours(a, w):
             xm[e, :int(cn[e])] = xp[int(of[e]):int(of[e]) + int(cn[e])]
         hm = torch.empty((E, cap, w.d_ff), dtype=w.w_dtype, device=dev)
         ym = torch.empty((E, cap, w.d), dtype=w.w_dtype, device=dev)
-
-        def mstep():
-            moe.moe_grouped_swiglu_masked(xm, D["W_gate"], D["W_up"], D["W_down"], counts, hm, ym, dev_status=status)
-
-        for _ in range(a.warmup):
-            mstep()
-        barrier()
-        m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        m0.record()
-        for _ in range(a.steps):
-            mstep()
-        m1.record()
-        torch.cuda.synchronize()
-        if status.item() != 0:
-            raise RuntimeError(f"device status {status.item()} in the masked-layout timing")
-        mms = m0.elapsed_time(m1) / a.steps
+        ms, _, _ = _timed(lambda: moe.moe_grouped_swiglu_masked(xm, D["W_gate"], D["W_up"], D["W_down"], counts, hm,
+                                                                ym, dev_status=status), a.steps, a.warmup, barrier)
+        L.check_status("in the masked-layout timing")
+        mms = ms / a.steps
         mbytes = active * 3 * w.d_ff * w.d * esz + S * (2 * w.d + 2 * w.d_ff) * esz
-        masked = {"expert_mlp_ms": mms, "tokens_per_s": T / (mms / 1000.0), "cap": cap,
-                  "hbm_achieved_gbs": mbytes / (mms / 1000.0) / 1e9,
-                  "hbm_frac": mbytes / (mms / 1000.0) / 1e9 / pk["hbm_gbs"], "algorithmic_bytes": mbytes,
-                  "contiguous_expert_mlp_ms": stage_ms["gate_up"] + stage_ms["down"]}
+        res["masked_layout"] = {"expert_mlp_ms": mms, "tokens_per_s": T / (mms / 1000.0), "cap": cap,
+                                "hbm_achieved_gbs": mbytes / (mms / 1000.0) / 1e9,
+                                "hbm_frac": mbytes / (mms / 1000.0) / 1e9 / pk["hbm_gbs"],
+                                "algorithmic_bytes": mbytes}
+        del xm, hm, ym
 
-    # ---- the layer with block-FP8 experts (weights quantised on the device beforehand)
-    fp8 = None
     if not a.no_fp8 and w.w_dtype == torch.bfloat16 and S // E <= 32:
         Wq = [moe.quantize_fp8_weights(D[n]) for n in ("W_gate", "W_up", "W_down")]
-        out8 = torch.empty_like(out)
+        out8 = torch.empty_like(L.out)
         ws8 = torch.empty(moe.forward_fp8_workspace_bytes(D["x"], D["W_r"], Wq[0][0], out8, k, w.eps),
                           dtype=torch.uint8, device=dev)
-
-        def fstep():
-            moe.moe_forward_fp8(D["x"], D["gamma"], D["W_r"], D["b"], *Wq, out8, top_k=k, eps=w.eps, ws=ws8,
-                                dev_status=status)
-
-        for _ in range(a.warmup):
-            fstep()
-        barrier()
-        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        g0.record()
-        for _ in range(a.steps):
-            fstep()
-        g1.record()
-        torch.cuda.synchronize()
-        if status.item() != 0:
-            raise RuntimeError(f"device status {status.item()} in the FP8 timing")
-        fms = g0.elapsed_time(g1) / a.steps
+        ms, _, _ = _timed(lambda: moe.moe_forward_fp8(D["x"], D["gamma"], D["W_r"], D["b"], *Wq, out8, top_k=k,
+                                                      eps=w.eps, ws=ws8, dev_status=status),
+                          a.steps, a.warmup, barrier)
+        L.check_status("in the FP8 timing")
+        fms = ms / a.steps
         # algorithmic bytes: active experts' codes and scales, the input, the output and the router weights
         fbytes = active * 3 * w.d_ff * w.d * (1 + 4 / (128 * 128)) + T * w.d * (D["x"].element_size() +
-                                                                                 out.element_size()) + E * w.d * 4
-        fp8 = {"ms_per_step": fms, "tokens_per_s": T / (fms / 1000.0), "dtype": "e4m3 experts, fp32 router",
-               "algorithmic_bytes": fbytes, "hbm_achieved_gbs": fbytes / (fms / 1000.0) / 1e9,
-               "hbm_frac": fbytes / (fms / 1000.0) / 1e9 / pk["hbm_gbs"],
-               "vs_bf16_layer": ms_per_step / fms}
-        del Wq
+                                                                                 L.out.element_size()) + E * w.d * 4
+        res["fp8_layer"] = {"ms_per_step": fms, "tokens_per_s": T / (fms / 1000.0),
+                            "dtype": "e4m3 experts, fp32 router", "algorithmic_bytes": fbytes,
+                            "hbm_achieved_gbs": fbytes / (fms / 1000.0) / 1e9,
+                            "hbm_frac": fbytes / (fms / 1000.0) / 1e9 / pk["hbm_gbs"],
+                            "vs_bf16_layer": ms_per_step / fms}
+        del Wq, ws8
 
-    # ---- expert parallelism with the exchange fused into the dispatch and combine kernels: one rank's step
-    epp = None
-    if not a.no_ep and world == 1 and w.w_dtype == torch.bfloat16:
+    if not a.no_ep and w.w_dtype == torch.bfloat16:
         from moe_layer_forward_b200 import ep_p2p
 
         peers = ep_p2p.local_peers(1, ep_p2p.capacity_rows(T, 1, k, E), w.d, w.w_dtype, dev)
-
-        def estep():
-            return ep_p2p.ep_p2p_forward_emulated([D["x"]], D["gamma"], D["W_r"], D["b"], D["W_gate"], D["W_up"],
-                                                  D["W_down"], top_k=k, eps=w.eps, peers=peers)
-
-        for _ in range(a.warmup):
-            estep()
-        barrier()
-        p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        p0.record()
-        for _ in range(a.steps):
-            estep()
-        p1.record()
-        torch.cuda.synchronize()
-        ems = p0.elapsed_time(p1) / a.steps
-        epp = {"ranks": 1, "ms_per_step": ems, "tokens_per_s": T / (ems / 1000.0), "vs_moe_forward": ms_per_step / ems,
-               "steps": "routing, permutation maps, dispatch into the receive buffer, layout, grouped MLP over "
-                        "the whole buffer, pull combine; no host synchronisation",
-               "multi_gpu": "not measured (one GPU per call here)"}
+        ms, _, _ = _timed(lambda: ep_p2p.ep_p2p_forward_emulated([D["x"]], D["gamma"], D["W_r"], D["b"], D["W_gate"],
+                                                                 D["W_up"], D["W_down"], top_k=k, eps=w.eps,
+                                                                 peers=peers), a.steps, a.warmup, barrier)
+        ems = ms / a.steps
+        res["ep_p2p"] = {"ranks": 1, "ms_per_step": ems, "tokens_per_s": T / (ems / 1000.0),
+                         "vs_moe_forward": ms_per_step / ems,
+                         "steps": "routing, permutation maps, dispatch into the receive buffer, layout, grouped MLP "
+                                  "over the whole buffer, pull combine; no host synchronisation",
+                         "multi_gpu": "not measured (one GPU per call here)"}
         del peers
+    return res
 
-    # ---- end to end through the public API with host buffers
-    e2e = None
-    if not a.no_e2e:
-        x_host = I["x"].pin_memory()
-        out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        x_dev = torch.empty_like(D["x"])
-        for _ in range(a.warmup):
-            x_dev.copy_(x_host, non_blocking=True)
-            step(x_dev)
-            out_host.copy_(out, non_blocking=True)
-            torch.cuda.current_stream().synchronize()
-        barrier()
-        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        f0.record()
-        for _ in range(a.steps):
-            x_dev.copy_(x_host, non_blocking=True)
-            step(x_dev)
-            out_host.copy_(out, non_blocking=True)
-            torch.cuda.current_stream().synchronize()  # the host reads this step's result
-        f1.record()
-        barrier()
-        e2e_value, _ = aggregate(f0.elapsed_time(f1), T, a.steps, world, max_over_ranks)
-        e2e = {"value": e2e_value, "unit": "tokens/s",
-               "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
-               "d2h_bytes_per_step": out_host.numel() * out_host.element_size()}
 
-    cpu = None
+def measure_workload(a, w, dev, world, rank, local, barrier, max_over_ranks, headline: bool) -> dict:
+    """Everything the bench reports for one workload: the timed layer, its roofline fractions, the stage
+    breakdown and dominant kernel, near-tie tokens, end-to-end throughput and the CPU oracle sample."""
+    import torch
+
+    pk = peaks()
+    L = Layer(w, dev)
+    L.step()
+    torch.cuda.synchronize()
+    L.check_status("after the first step")
+    ms, clk, launches = _timed(L.step, a.steps, a.warmup, barrier, clocks_gpu=local)
+    value, ms_per_step = aggregate(ms, w.T, a.steps, world, max_over_ranks)
+    L.check_status("in the timed region")
+    stage_ms, kroof, active, bufs = staged(L, a, barrier, pk)
+    r = {"workload": w.name, "ms_per_step": ms_per_step, "tokens_per_s": value, "steps": a.steps,
+         "warmup": a.warmup, "gpu_launches": launches, "clocks": clk, "active_experts": active,
+         "layer_roofline": layer_roofline(w, active, ms_per_step, pk), "dominant_kernel": kroof,
+         "stages_ms": stage_ms, "near_ties": near_ties(L), "config": config_of(w, world)}
+    r["e2e"] = None if a.no_e2e else e2e_of(L, a, barrier, world, max_over_ranks)
+    if headline:
+        r.update(headline_extras(L, a, barrier, pk, ms_per_step, bufs, active))
+    r["cpu_baseline"] = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        cpu = cpu_baseline(I, w)
+        r["cpu_baseline"] = cpu_baseline(L.I, w, seconds=15.0 if headline else 10.0)
+    del L, bufs
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return r
+
+
+def run_ours(a, w):
+    import torch
+    import torch.distributed as dist
+
+    import synth
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    max_over_ranks = reduce_max_fn(dist, dev)
+    # the headline workload first; at one GPU the other four workloads follow, one at a time (each freed
+    # before the next is built); under torchrun every rank measures the headline workload only
+    names = [w.name]
+    if world == 1 and a.workloads == "all" and a.shrink == 1:
+        names += [n for n in synth.WORKLOADS if n != w.name]
+    results = {}
+    for n in names:
+        wl = w if n == w.name else synth.WORKLOADS[n]
+        results[n] = measure_workload(a, wl, dev, world, rank, local, barrier, max_over_ranks, headline=(n == w.name))
+    h = results[w.name]
 
     if rank == 0:
-        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": a.steps,
-                "warmup": a.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "bf16" if w.w_dtype == torch.bfloat16 else "f32",
-                "data": "synthetic", "config": config_of(w, world), "roofline": roof, "cpu_baseline": cpu,
-                "e2e": e2e, "gpu_launches": launches, "clocks": clk.summary(),
-                "stages_ms": stage_ms, "active_experts": active, "masked_layout": masked, "fp8_layer": fp8,
-                "ep_p2p": epp}
+        line = {"metric": METRIC, "value": h["tokens_per_s"], "unit": "tokens/s", "n_gpus": world,
+                "steps": a.steps, "warmup": a.warmup, "ms_per_step": h["ms_per_step"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.w_dtype == torch.bfloat16 else "f32",
+                "data": "synthetic", "config": h["config"], "roofline": h["dominant_kernel"],
+                "layer_roofline": h["layer_roofline"], "cpu_baseline": h["cpu_baseline"], "e2e": h["e2e"],
+                "gpu_launches": h["gpu_launches"], "clocks": h["clocks"], "stages_ms": h["stages_ms"],
+                "active_experts": h["active_experts"], "near_ties": h["near_ties"],
+                "masked_layout": h.get("masked_layout"), "fp8_layer": h.get("fp8_layer"), "ep_p2p": h.get("ep_p2p")}
+        if len(results) > 1:
+            keep = ("ms_per_step", "tokens_per_s", "layer_roofline", "dominant_kernel", "stages_ms", "near_ties",
+                    "active_experts", "clocks", "gpu_launches", "e2e", "cpu_baseline", "config")
+            line["workloads"] = {n: {k: r[k] for k in keep} for n, r in results.items()}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

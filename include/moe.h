@@ -56,7 +56,7 @@ typedef enum {
 /* bits OR-ed into *dev_status by kernels */
 #define MOE_DEV_BAD_EXPERT_ID 1 /* topk_idx held an id outside [0, E); that pair was dropped */
 #define MOE_DEV_TIMEOUT 2       /* a bounded in-kernel wait gave up; outputs are not valid */
-#define MOE_DEV_BAD_COUNT 4     /* a masked-layout count was outside [0, cap]; it was clamped */
+#define MOE_DEV_BAD_COUNT 4     /* a row count or offset disagreed with the buffers; see each call */
 
 #define MOE_MAX_EXPERTS 256
 #define MOE_MAX_TOP_K 8
@@ -156,7 +156,8 @@ moe_status_t moe_permute(const void* v, moe_dtype_t v_dt, const int32_t* topk_id
  *     MOE_ERR_UNSUPPORTED; other arguments as for moe_permute.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     before any stream capture.  A lookup that fails returns MOE_ERR_CUDA and
+ *     is tried again by the next call.
  *   - All calls share the one array and nothing in it needs to start at zero
  *     (every entry read is written earlier in the same call), but calls whose
  *     work overlaps on the GPU (other streams, other host threads) race on it:
@@ -175,7 +176,12 @@ moe_status_t moe_permute_static_ws(const void* v, moe_dtype_t v_dt, const int32_
  * SiLU(x) = x * sigmoid(x).  dt = MOE_BF16: tcgen05 tensor cores, fp32
  * accumulation in tensor memory, h rounded to bf16; dt = MOE_F32: fp32 CUDA cores.
  * xp [S][d], h [S][d_ff] (dtype dt); counts/offsets as written by moe_permute.
- * Rows outside every segment are not written.
+ * Rows outside every segment are not written.  A segment that does not fit the
+ * S rows (negative count or offset, or offsets[e] + counts[e] > S) is clamped
+ * into them and sets MOE_DEV_BAD_COUNT, so no row outside [0, S) is read or
+ * written whatever the device-side counts hold.  (The same holds for
+ * moe_expert_down, moe_grouped_swiglu, moe_grouped_swiglu_sized with S_cap
+ * rows, and moe_grouped_swiglu_fp8.)
  * bf16 requires d % 64 == 0, d_ff % 128 == 0, 16-byte aligned pointers.
  */
 moe_status_t moe_expert_gate_up(const void* xp, const void* W_gate, const void* W_up, moe_dtype_t dt,
@@ -239,7 +245,9 @@ moe_status_t moe_grouped_swiglu_masked(const void* x, const void* W_gate, const 
  * Step 5 — weighted un-permute and residual [P1 §EP 路径: weighted sum at the
  * source; §Norm&Residual: X' = R + FFN(V); P5 token_unpermutation]:
  *   out[t][j] = residual[t][j] + sum_{i<k} topk_w[t][i] * y[token_slot[t][i]][j]
- * fp32 accumulation in pick order.  Picks with token_slot == -1 are skipped.
+ * fp32 accumulation in pick order.  Picks with a negative token_slot (moe_permute
+ * writes -1 for a bad expert id) are skipped: their row is not read and their
+ * weight takes no part.
  * y [T*k][d] (y_dt), residual [T][d] (r_dt), out [T][d] (out_dt).
  * Requires d % 8 == 0 and 16-byte aligned y, residual, out.
  */
@@ -330,29 +338,38 @@ moe_status_t moe_forward_fp8(const moe_shape_t* shape, const moe_weights_fp8_t* 
  * its receive buffer; all expert MLPs complete before any combine reads their
  * outputs).  Requires E % N == 0, N <= MOE_MAX_EP_RANKS, d % 8 == 0.
  *
+ * recv_rows is the row count of every rank's receive / output buffer (the
+ * same on all ranks); no row at or past it is stored or loaded.
+ *
  * moe_ep_dispatch: the permutation's row copy to the owners: for every pick
  *   (t, i) of this rank with expert e = topk_idx[t][i] and slot
  *   s = token_slot[t][i], recv_bufs[e / (E/N)][row(rank, e, s - offsets[e])] = v[t].
  *   topk_idx / token_slot / offsets as returned by moe_router_topk and
- *   moe_permute on this rank.  A bad pick sets MOE_DEV_BAD_EXPERT_ID.
+ *   moe_permute on this rank.  A pick with a bad expert id or slot sets
+ *   MOE_DEV_BAD_EXPERT_ID; a pick whose index inside its segment is outside
+ *   [0, count_table[rank][e]) or whose row falls outside [0, recv_rows) (a
+ *   table that disagrees with the routing, or a short buffer) is not stored
+ *   and sets MOE_DEV_BAD_COUNT.
  * moe_ep_layout: counts_loc[e] = sum_s count_table[s][rank E/N + e] and
  *   offsets_loc[0 .. E/N] its exclusive prefix (the receive buffer's segments).
  * moe_ep_combine: step 5 with each pick's expert output row read from its
  *   owner: out[t] = residual[t] + sum_{i<k} topk_w[t][i] * y_bufs[owner][row]
- *   in fp32, pick order; the same arithmetic as moe_unpermute_combine.
+ *   in fp32, pick order; the same arithmetic as moe_unpermute_combine.  A
+ *   pick that fails the dispatch's checks is left out of the sum (its row is
+ *   not read) and sets the same status bit.
  */
 #define MOE_MAX_EP_RANKS 64
 moe_status_t moe_ep_dispatch(const void* v, moe_dtype_t v_dt, const int32_t* topk_idx, const int32_t* token_slot,
                              const int32_t* offsets, const int32_t* count_table, int32_t rank, int32_t N, int32_t E,
-                             int32_t T, int32_t d, int32_t k, void* const* recv_bufs, int32_t* dev_status,
-                             moe_stream_t stream);
+                             int32_t T, int32_t d, int32_t k, void* const* recv_bufs, int64_t recv_rows,
+                             int32_t* dev_status, moe_stream_t stream);
 moe_status_t moe_ep_layout(const int32_t* count_table, int32_t rank, int32_t N, int32_t E, int32_t* counts_loc,
                            int32_t* offsets_loc, moe_stream_t stream);
 moe_status_t moe_ep_combine(const void* const* y_bufs, moe_dtype_t y_dt, const int32_t* topk_idx,
                             const int32_t* token_slot, const int32_t* offsets, const int32_t* count_table,
                             int32_t rank, int32_t N, int32_t E, const float* topk_w, const void* residual,
                             moe_dtype_t r_dt, int32_t T, int32_t d, int32_t k, void* out, moe_dtype_t out_dt,
-                            int32_t* dev_status, moe_stream_t stream);
+                            int64_t recv_rows, int32_t* dev_status, moe_stream_t stream);
 
 /* Number of kernels the library has enqueued in this process since it was
  * loaded, over all entry points, streams and threads (successful launches
@@ -362,7 +379,7 @@ moe_status_t moe_ep_combine(const void* const* y_bufs, moe_dtype_t y_dt, const i
 uint64_t moe_kernel_launches(void);
 
 /* ABI version of this header (bumped on any incompatible change). */
-#define MOE_ABI_VERSION 1
+#define MOE_ABI_VERSION 2
 int32_t moe_abi_version(void);
 
 #ifdef __cplusplus

@@ -64,10 +64,10 @@ _sig = {
                         _vp, _vp],
     "moe_grouped_swiglu_sized": [_vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp,
                                  _vp],
-    "moe_ep_dispatch": [_vp, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp],
+    "moe_ep_dispatch": [_vp, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp],
     "moe_ep_layout": [_vp, _i32, _i32, _i32, _vp, _vp, _vp],
     "moe_ep_combine": [_vp, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _i32,
-                       _vp, _vp],
+                       _i64, _vp, _vp],
 }
 for _name, _args in _sig.items():
     _fn = getattr(_lib, _name)
@@ -227,16 +227,17 @@ def moe_grouped_swiglu_sized(xp, W_gate, W_up, W_down, counts, offsets, h, y, S_
 
 
 # --------------------------------------------------------------------------- expert parallelism over peer memory
-def moe_ep_dispatch(v, topk_idx, token_slot, offsets, count_table, rank: int, recv_ptrs, dev_status=None) -> None:
+def moe_ep_dispatch(v, topk_idx, token_slot, offsets, count_table, rank: int, recv_ptrs, recv_rows: int,
+                    dev_status=None) -> None:
     """Store this rank's routed rows of v into their owners' receive buffers.
 
     count_table: int32 [N][E] on the device (every rank's counts); recv_ptrs: int64 [N] on the device, the
-    receive buffers' addresses as mapped into this process."""
+    receive buffers' addresses as mapped into this process; recv_rows: rows of every receive buffer."""
     T, d = v.shape
     k = topk_idx.shape[1]
     N, E = count_table.shape
     _check("moe_ep_dispatch", _lib.moe_ep_dispatch(_p(v), _dt(v), _p(topk_idx), _p(token_slot), _p(offsets),
-                                                   _p(count_table), rank, N, E, T, d, k, _p(recv_ptrs),
+                                                   _p(count_table), rank, N, E, T, d, k, _p(recv_ptrs), recv_rows,
                                                    _p(dev_status), _stream(v.device)))
 
 
@@ -248,18 +249,19 @@ def moe_ep_layout(count_table, rank: int, counts_loc, offsets_loc) -> None:
 
 
 def moe_ep_combine(y_ptrs, y_dtype, topk_idx, token_slot, offsets, count_table, rank: int, topk_w, residual, out,
-                   dev_status=None) -> None:
+                   recv_rows: int, dev_status=None) -> None:
     """out = residual + sum_i w_i y_i with each pick's row y_i read from its owner's output buffer.
 
-    y_ptrs: int64 [N] on the device, the expert output buffers' addresses; y_dtype their torch dtype."""
+    y_ptrs: int64 [N] on the device, the expert output buffers' addresses; y_dtype their torch dtype;
+    recv_rows: rows of every output buffer."""
     T, d = residual.shape
     k = topk_idx.shape[1]
     N, E = count_table.shape
     ydt = MOE_BF16 if y_dtype == torch.bfloat16 else MOE_F32
     _check("moe_ep_combine", _lib.moe_ep_combine(_p(y_ptrs), ydt, _p(topk_idx), _p(token_slot), _p(offsets),
                                                  _p(count_table), rank, N, E, _p(topk_w), _p(residual),
-                                                 _dt(residual), T, d, k, _p(out), _dt(out), _p(dev_status),
-                                                 _stream(residual.device)))
+                                                 _dt(residual), T, d, k, _p(out), _dt(out), recv_rows,
+                                                 _p(dev_status), _stream(residual.device)))
 
 
 def _shape(x, W_gate, out, top_k, eps, E) -> MoeShape:

@@ -202,7 +202,7 @@ moe_status_t moe_expert_gate_up(const void* xp, const void* W_gate, const void* 
         return cuda_status(launch_gate_up_bf16(c, xp, W_gate, W_up, counts, offsets, S, E, d, d_ff, h, dev_status));
     return cuda_status(launch_gate_up_f32(c, static_cast<const float*>(xp), static_cast<const float*>(W_gate),
                                           static_cast<const float*>(W_up), counts, offsets, S, E, d, d_ff,
-                                          static_cast<float*>(h)));
+                                          static_cast<float*>(h), dev_status));
 }
 
 moe_status_t moe_expert_down(const void* h, const void* W_down, moe_dtype_t dt, const int32_t* counts,
@@ -218,7 +218,7 @@ moe_status_t moe_expert_down(const void* h, const void* W_down, moe_dtype_t dt, 
     if (st != MOE_OK) return st;
     if (dt == MOE_BF16) return cuda_status(launch_down_bf16(c, h, W_down, counts, offsets, S, E, d, d_ff, y, dev_status));
     return cuda_status(launch_down_f32(c, static_cast<const float*>(h), static_cast<const float*>(W_down), counts,
-                                       offsets, S, E, d, d_ff, static_cast<float*>(y)));
+                                       offsets, S, E, d, d_ff, static_cast<float*>(y), dev_status));
 }
 
 moe_status_t moe_grouped_swiglu(const void* xp, const void* W_gate, const void* W_up, const void* W_down,
@@ -255,10 +255,10 @@ moe_status_t moe_grouped_swiglu_sized(const void* xp, const void* W_gate, const 
     }
     st = cuda_status(launch_gate_up_f32(c, static_cast<const float*>(xp), static_cast<const float*>(W_gate),
                                         static_cast<const float*>(W_up), counts, offsets, S_cap, E, d, d_ff,
-                                        static_cast<float*>(h)));
+                                        static_cast<float*>(h), dev_status));
     if (st != MOE_OK) return st;
     return cuda_status(launch_down_f32(c, static_cast<const float*>(h), static_cast<const float*>(W_down), counts,
-                                       offsets, S_cap, E, d, d_ff, static_cast<float*>(y)));
+                                       offsets, S_cap, E, d, d_ff, static_cast<float*>(y), dev_status));
 }
 
 moe_status_t moe_grouped_swiglu_masked(const void* x, const void* W_gate, const void* W_up, const void* W_down,
@@ -309,9 +309,9 @@ moe_status_t check_ep(int32_t rank, int32_t N, int32_t E, int32_t T, int32_t d, 
 
 moe_status_t moe_ep_dispatch(const void* v, moe_dtype_t v_dt, const int32_t* topk_idx, const int32_t* token_slot,
                              const int32_t* offsets, const int32_t* count_table, int32_t rank, int32_t N, int32_t E,
-                             int32_t T, int32_t d, int32_t k, void* const* recv_bufs, int32_t* dev_status,
-                             moe_stream_t stream) {
-    if (!valid_dt(v_dt)) return MOE_ERR_INVALID_ARG;
+                             int32_t T, int32_t d, int32_t k, void* const* recv_bufs, int64_t recv_rows,
+                             int32_t* dev_status, moe_stream_t stream) {
+    if (!valid_dt(v_dt) || recv_rows < 0) return MOE_ERR_INVALID_ARG;
     moe_status_t st = check_ep(rank, N, E, T, d, k, count_table);
     if (st != MOE_OK) return st;
     if (T == 0) return MOE_OK;
@@ -320,7 +320,7 @@ moe_status_t moe_ep_dispatch(const void* v, moe_dtype_t v_dt, const int32_t* top
     st = make_ctx(stream, c);
     if (st != MOE_OK) return st;
     return cuda_status(launch_ep_dispatch(c, v, v_dt, topk_idx, token_slot, offsets, count_table, rank, N, E, T, d, k,
-                                          recv_bufs, dev_status));
+                                          recv_bufs, recv_rows, dev_status));
 }
 
 moe_status_t moe_ep_layout(const int32_t* count_table, int32_t rank, int32_t N, int32_t E, int32_t* counts_loc,
@@ -338,8 +338,8 @@ moe_status_t moe_ep_combine(const void* const* y_bufs, moe_dtype_t y_dt, const i
                             const int32_t* token_slot, const int32_t* offsets, const int32_t* count_table,
                             int32_t rank, int32_t N, int32_t E, const float* topk_w, const void* residual,
                             moe_dtype_t r_dt, int32_t T, int32_t d, int32_t k, void* out, moe_dtype_t out_dt,
-                            int32_t* dev_status, moe_stream_t stream) {
-    if (!valid_dt(y_dt) || !valid_dt(r_dt) || !valid_dt(out_dt)) return MOE_ERR_INVALID_ARG;
+                            int64_t recv_rows, int32_t* dev_status, moe_stream_t stream) {
+    if (!valid_dt(y_dt) || !valid_dt(r_dt) || !valid_dt(out_dt) || recv_rows < 0) return MOE_ERR_INVALID_ARG;
     moe_status_t st = check_ep(rank, N, E, T, d, k, count_table);
     if (st != MOE_OK) return st;
     if (T == 0) return MOE_OK;
@@ -349,7 +349,7 @@ moe_status_t moe_ep_combine(const void* const* y_bufs, moe_dtype_t y_dt, const i
     st = make_ctx(stream, c);
     if (st != MOE_OK) return st;
     return cuda_status(launch_ep_combine(c, y_bufs, y_dt, topk_idx, token_slot, offsets, count_table, rank, N, E,
-                                         topk_w, residual, r_dt, T, d, k, out, out_dt, dev_status));
+                                         topk_w, residual, r_dt, T, d, k, out, out_dt, recv_rows, dev_status));
 }
 
 moe_status_t moe_forward(const moe_shape_t* shape, const moe_weights_t* wts, const void* x, void* out,
@@ -433,10 +433,10 @@ moe_status_t moe_forward(const moe_shape_t* shape, const moe_weights_t* wts, con
     } else {
         st = cuda_status(launch_gate_up_f32(c, static_cast<const float*>(xp), static_cast<const float*>(wts->W_gate),
                                             static_cast<const float*>(wts->W_up), counts, offsets, S, E, d, d_ff,
-                                            static_cast<float*>(h)));
+                                            static_cast<float*>(h), dev_status));
         if (st != MOE_OK) return st;
         st = cuda_status(launch_down_f32(c, static_cast<const float*>(h), static_cast<const float*>(wts->W_down),
-                                         counts, offsets, S, E, d, d_ff, static_cast<float*>(y)));
+                                         counts, offsets, S, E, d, d_ff, static_cast<float*>(y), dev_status));
     }
     if (st != MOE_OK) return st;
     // 5. weighted un-permute + residual
@@ -481,7 +481,7 @@ moe_status_t moe_grouped_swiglu_fp8(const uint8_t* xq, const float* xs, const mo
     st = make_ctx(stream, c);
     if (st != MOE_OK) return st;
     st = cuda_status(launch_gate_up_fp8(c, xq, xs, nullptr, w->W_gate_q, w->W_gate_s, w->W_up_q, w->W_up_s, counts,
-                                        offsets, S, E, d, d_ff, hq, hs, dev_status));
+                                        offsets, S, E, d, d_ff, hq, hs, dev_status, S));
     if (st != MOE_OK) return st;
     return cuda_status(
         launch_down_fp8(c, hq, hs, w->W_down_q, w->W_down_s, counts, offsets, S, E, d, d_ff, y, dev_status));
@@ -553,7 +553,7 @@ moe_status_t moe_forward_fp8(const moe_shape_t* shape, const moe_weights_fp8_t* 
     if (st != MOE_OK) return st;
     // 4. block-FP8 SwiGLU MLP
     st = cuda_status(launch_gate_up_fp8(c, vq, vs, slot_token, w->W_gate_q, w->W_gate_s, w->W_up_q, w->W_up_s, counts,
-                                        offsets, S, E, d, d_ff, hq, hs, dev_status));
+                                        offsets, S, E, d, d_ff, hq, hs, dev_status, T));
     if (st != MOE_OK) return st;
     st = cuda_status(
         launch_down_fp8(c, hq, hs, w->W_down_q, w->W_down_s, counts, offsets, S, E, d, d_ff, y, dev_status));

@@ -6,6 +6,9 @@
 //
 //   out[t][j] = residual[t][j] + sum_{i<k} w[t][i] * y[token_slot[t][i]][j]
 //
+// A pick whose slot is negative (the permutation marks a pick with a bad
+// expert id that way) is skipped: neither its row is read nor its weight used.
+//
 // One warp owns a (token, 256-column segment) unit: lanes below k load the
 // token's k slots and weights once and broadcast them by shuffle; each lane
 // then gathers its 8 columns from the k expert rows (16-byte loads, all
@@ -48,7 +51,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const void* __restrict__ y
         uint4 raw[kMaxTopK][V];
 #pragma unroll
         for (int i = 0; i < kMaxTopK; ++i) {
-            if (i < k) {
+            if (i < k && slot[i] >= 0) {
                 const int64_t e0 = (int64_t)slot[i] * d + j;
 #pragma unroll
                 for (int v = 0; v < V; ++v)
@@ -61,7 +64,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const void* __restrict__ y
         for (int q = 0; q < 8; ++q) acc[q] = 0.f;
 #pragma unroll
         for (int i = 0; i < kMaxTopK; ++i) {
-            if (i < k) {
+            if (i < k && slot[i] >= 0) {
                 float yv[8];
                 if constexpr (YDT == DT_BF16) {
                     const uint32_t wv[4] = {raw[i][0].x, raw[i][0].y, raw[i][0].z, raw[i][0].w};

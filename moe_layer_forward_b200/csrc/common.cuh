@@ -70,4 +70,17 @@ __device__ __forceinline__ void set_status(int32_t* status, int bits) {
     if (status) atomicOr(status, bits);
 }
 
+// Expert segment [off, off + cnt) as given, cut to the rows [0, S) of the buffer: (o, n) is the
+// intersection.  Returns false when the given segment does not lie inside the buffer (negative count or
+// offset, or past its end); the caller flags DEV_BAD_COUNT.
+__device__ __forceinline__ bool clamp_segment(int off, int cnt, int S, int& o, int& n) {
+    const bool ok = off >= 0 && cnt >= 0 && (int64_t)off + cnt <= (int64_t)S;
+    const int64_t lo = off < 0 ? 0 : (off > S ? S : off);
+    int64_t hi = cnt < 0 ? lo : (int64_t)off + cnt;
+    if (hi > S) hi = S;
+    o = (int)lo;
+    n = hi > lo ? (int)(hi - lo) : 0;
+    return ok;
+}
+
 }  // namespace moe

@@ -86,11 +86,13 @@ __global__ void __launch_bounds__(256) ep_dispatch_kernel(const uint8_t* __restr
                                                           const int32_t* __restrict__ offsets,
                                                           const int32_t* __restrict__ table, int rank, int N, int E,
                                                           int T, int k, uint8_t* const* __restrict__ recv,
-                                                          int32_t* status) {
-    __shared__ int dbase[kMaxExperts], scratch[kMaxExperts];
+                                                          int64_t recv_rows, int32_t* status) {
+    __shared__ int dbase[kMaxExperts], scratch[kMaxExperts], own[kMaxExperts];
     pdl_wait();
     pdl_trigger();
     ep_dest_base(table, rank, N, E, dbase, scratch);
+    for (int e = threadIdx.x; e < E; e += blockDim.x) own[e] = table[(int64_t)rank * E + e];
+    __syncthreads();
     const int E_loc = E / N;
     const int64_t cpr = row_bytes / 16;
     const int64_t n = (int64_t)T * cpr;
@@ -106,7 +108,14 @@ __global__ void __launch_bounds__(256) ep_dispatch_kernel(const uint8_t* __restr
                 if (c == 0) set_status(status, DEV_BAD_EXPERT_ID);
                 continue;
             }
-            const int64_t row = (int64_t)dbase[e] + (s - offsets[e]);
+            // the row must lie in this rank's part of e's segment and inside the receive buffer: a table
+            // that disagrees with the routing (or a short buffer) skips the store and is reported
+            const int i_e = s - offsets[e];
+            const int64_t row = (int64_t)dbase[e] + i_e;
+            if (i_e < 0 || i_e >= own[e] || row < 0 || row >= recv_rows) {
+                if (c == 0) set_status(status, DEV_BAD_COUNT);
+                continue;
+            }
             st16(recv[e / E_loc] + row * row_bytes + c * 16, val);
         }
     }
@@ -148,11 +157,13 @@ __global__ void __launch_bounds__(256) ep_combine_kernel(const void* const* __re
                                                          const int32_t* __restrict__ table, int rank, int N, int E,
                                                          const float* __restrict__ w, const void* __restrict__ res,
                                                          int T, int d, int k, void* __restrict__ out,
-                                                         int32_t* status) {
-    __shared__ int dbase[kMaxExperts], scratch[kMaxExperts];
+                                                         int64_t recv_rows, int32_t* status) {
+    __shared__ int dbase[kMaxExperts], scratch[kMaxExperts], own[kMaxExperts];
     pdl_wait();
     pdl_trigger();
     ep_dest_base(table, rank, N, E, dbase, scratch);
+    for (int e = threadIdx.x; e < E; e += blockDim.x) own[e] = table[(int64_t)rank * E + e];
+    __syncthreads();
     const int E_loc = E / N;
     const int lane = threadIdx.x & 31;
     const int nseg = (d + 255) / 256;
@@ -166,33 +177,39 @@ __global__ void __launch_bounds__(256) ep_combine_kernel(const void* const* __re
         int my_owner = 0;
         int64_t my_row = 0;
         float my_w = 0.f;
+        int my_ok = 0;
         if (lane < k) {
             const int e = __ldg(idx + t * k + lane);
             const int s = __ldg(token_slot + t * k + lane);
             my_w = __ldg(w + t * k + lane);
             if (e >= 0 && e < E && s >= 0) {
+                const int i_e = s - offsets[e];
                 my_owner = e / E_loc;
-                my_row = (int64_t)dbase[e] + (s - offsets[e]);
-            } else {
-                my_w = 0.f;  // a bad pick contributes nothing (row 0 of rank 0 is read and weighted by 0)
-                if (u - t * nseg == 0) set_status(status, DEV_BAD_EXPERT_ID);
+                my_row = (int64_t)dbase[e] + i_e;
+                my_ok = i_e >= 0 && i_e < own[e] && my_row >= 0 && my_row < recv_rows;
+                if (!my_ok && u - t * nseg == 0) set_status(status, DEV_BAD_COUNT);
+            } else if (u - t * nseg == 0) {
+                set_status(status, DEV_BAD_EXPERT_ID);
             }
         }
+        // a pick that is not valid is skipped: its row is neither read nor weighted
         int owner[kMaxTopK];
         int64_t row[kMaxTopK];
         float wt[kMaxTopK];
+        bool ok[kMaxTopK];
 #pragma unroll
         for (int i = 0; i < kMaxTopK; ++i) {
             owner[i] = __shfl_sync(0xffffffffu, my_owner, i);
             row[i] = __shfl_sync(0xffffffffu, my_row, i);
             wt[i] = __shfl_sync(0xffffffffu, my_w, i);
+            ok[i] = __shfl_sync(0xffffffffu, my_ok, i) != 0;
         }
         if (j >= d) continue;
         constexpr int V = YDT == DT_BF16 ? 1 : 2;
         uint4 raw[kMaxTopK][V];
 #pragma unroll
         for (int i = 0; i < kMaxTopK; ++i) {
-            if (i < k) {
+            if (i < k && ok[i]) {
                 const uint8_t* p = static_cast<const uint8_t*>(ybuf[owner[i]]) + (row[i] * d + j) * ES;
 #pragma unroll
                 for (int vv = 0; vv < V; ++vv) raw[i][vv] = ld16_plain(p + 16 * vv);
@@ -203,7 +220,7 @@ __global__ void __launch_bounds__(256) ep_combine_kernel(const void* const* __re
         for (int q = 0; q < 8; ++q) acc[q] = 0.f;
 #pragma unroll
         for (int i = 0; i < kMaxTopK; ++i) {
-            if (i < k) {
+            if (i < k && ok[i]) {
                 float yv[8];
                 if constexpr (YDT == DT_BF16) {
                     const uint32_t wv[4] = {raw[i][0].x, raw[i][0].y, raw[i][0].z, raw[i][0].w};
@@ -232,7 +249,7 @@ __global__ void __launch_bounds__(256) ep_combine_kernel(const void* const* __re
 
 cudaError_t launch_ep_dispatch(const Ctx& c, const void* v, int v_dt, const int32_t* idx, const int32_t* token_slot,
                                const int32_t* offsets, const int32_t* table, int rank, int N, int E, int T, int d,
-                               int k, void* const* recv, int32_t* status) {
+                               int k, void* const* recv, int64_t recv_rows, int32_t* status) {
     if (T == 0) return cudaSuccess;
     const int64_t row_bytes = (int64_t)d * (v_dt == DT_BF16 ? 2 : 4);
     const int64_t n = (int64_t)T * (row_bytes / 16);
@@ -241,7 +258,7 @@ cudaError_t launch_ep_dispatch(const Ctx& c, const void* v, int v_dt, const int3
     if (blocks > cap) blocks = cap;
     return launch(ep_dispatch_kernel, dim3((unsigned)blocks), dim3(256), 0, c, static_cast<const uint8_t*>(v),
                   row_bytes, idx, token_slot, offsets, table, rank, N, E, T, k,
-                  reinterpret_cast<uint8_t* const*>(recv), status);
+                  reinterpret_cast<uint8_t* const*>(recv), recv_rows, status);
 }
 
 cudaError_t launch_ep_layout(const Ctx& c, const int32_t* table, int rank, int N, int E, int32_t* counts_loc,
@@ -253,18 +270,18 @@ template <int YDT, int RDT>
 static cudaError_t launch_ep_combine_o(const Ctx& c, dim3 g, const void* const* y, const int32_t* idx,
                                       const int32_t* ts, const int32_t* off, const int32_t* table, int rank, int N,
                                       int E, const float* w, const void* res, int T, int d, int k, void* out,
-                                      int out_dt, int32_t* status) {
+                                      int out_dt, int64_t recv_rows, int32_t* status) {
     if (out_dt == DT_BF16)
         return launch(ep_combine_kernel<YDT, RDT, DT_BF16>, g, dim3(256), 0, c, y, idx, ts, off, table, rank, N, E, w,
-                      res, T, d, k, out, status);
+                      res, T, d, k, out, recv_rows, status);
     return launch(ep_combine_kernel<YDT, RDT, DT_F32>, g, dim3(256), 0, c, y, idx, ts, off, table, rank, N, E, w, res,
-                  T, d, k, out, status);
+                  T, d, k, out, recv_rows, status);
 }
 
 cudaError_t launch_ep_combine(const Ctx& c, const void* const* y, int y_dt, const int32_t* idx,
                               const int32_t* token_slot, const int32_t* offsets, const int32_t* table, int rank, int N,
                               int E, const float* w, const void* res, int r_dt, int T, int d, int k, void* out,
-                              int out_dt, int32_t* status) {
+                              int out_dt, int64_t recv_rows, int32_t* status) {
     if (T == 0) return cudaSuccess;
     const int64_t n = (int64_t)T * ((d + 255) / 256);
     int64_t blocks = (n + 7) / 8;
@@ -273,15 +290,15 @@ cudaError_t launch_ep_combine(const Ctx& c, const void* const* y, int y_dt, cons
     const dim3 g((unsigned)blocks);
     if (y_dt == DT_BF16 && r_dt == DT_BF16)
         return launch_ep_combine_o<DT_BF16, DT_BF16>(c, g, y, idx, token_slot, offsets, table, rank, N, E, w, res, T,
-                                                     d, k, out, out_dt, status);
+                                                     d, k, out, out_dt, recv_rows, status);
     if (y_dt == DT_BF16)
         return launch_ep_combine_o<DT_BF16, DT_F32>(c, g, y, idx, token_slot, offsets, table, rank, N, E, w, res, T, d,
-                                                    k, out, out_dt, status);
+                                                    k, out, out_dt, recv_rows, status);
     if (r_dt == DT_BF16)
         return launch_ep_combine_o<DT_F32, DT_BF16>(c, g, y, idx, token_slot, offsets, table, rank, N, E, w, res, T, d,
-                                                    k, out, out_dt, status);
+                                                    k, out, out_dt, recv_rows, status);
     return launch_ep_combine_o<DT_F32, DT_F32>(c, g, y, idx, token_slot, offsets, table, rank, N, E, w, res, T, d, k,
-                                               out, out_dt, status);
+                                               out, out_dt, recv_rows, status);
 }
 
 }  // namespace moe

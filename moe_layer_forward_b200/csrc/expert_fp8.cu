@@ -261,7 +261,21 @@ struct Args {
     float* out_s;           //          h scales [S][n_out / 128]
     uint16_t* out;          // down:    y bf16 [S][n_out]
     int32_t* status;
+    int S;                  // rows of the expert-contiguous outputs; a segment that does not fit is clamped and flagged
+    int act_rows;           // rows of act when gather is set
 };
+
+// input row of expert-contiguous slot `slot`: the slot itself, or its entry of the gather map (a map
+// entry outside the input reads row 0 instead and is flagged)
+__device__ __forceinline__ int input_row(const Args& p, int slot) {
+    if (!p.gather) return slot;
+    const int t = p.gather[slot];
+    if (t < 0 || t >= p.act_rows) {
+        set_status(p.status, DEV_BAD_COUNT);
+        return 0;
+    }
+    return t;
+}
 
 struct Aux {
     uint64_t full[8];
@@ -325,8 +339,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     pdl_wait();
     const int E = p.E;
     for (int e = threadIdx.x; e < E; e += kThreads) {
-        aux.cnt[e] = p.counts[e];
-        aux.off[e] = p.offsets[e];
+        int o, n;
+        if (!clamp_segment(p.offsets[e], p.counts[e], p.S, o, n)) set_status(p.status, DEV_BAD_COUNT);
+        aux.cnt[e] = n;
+        aux.off[e] = o;
     }
     __syncthreads();
     if (warp == 0) {
@@ -464,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < RPL; ++i) {
                     const int r = r0 + 4 * i;
-                    src_row[i] = r < rows ? (p.gather ? p.gather[base + r] : base + r) : 0;
+                    src_row[i] = r < rows ? input_row(p, base + r) : 0;
                 }
                 cur = tile;
             }
@@ -500,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int rows = min(R, aux.cnt[e] - rb * R);
             const int base = aux.off[e] + rb * R;
             // lane n < rows: input row of token column n (its activation scales)
-            const int my_row = lane < rows ? (p.gather ? p.gather[base + lane] : base + lane) : 0;
+            const int my_row = lane < rows ? input_row(p, base + lane) : 0;
             // weight scale rows: gate and up of block cb, or down blocks NA*cb (and NA*cb + 1)
             const int64_t wb = (int64_t)e * (p.n_out / 128) + (SWIGLU ? cb : NA * cb);
             const float* s1 = p.w1_s + wb * nk;
@@ -658,9 +674,10 @@ static int fp8_rows(int S, int E) { return E > 0 && S / E <= 8 ? 16 : 32; }
 cudaError_t launch_gate_up_fp8(const Ctx& c, const uint8_t* xq, const float* xs, const int32_t* gather,
                                const uint8_t* Wg, const float* Wg_s, const uint8_t* Wu, const float* Wu_s,
                                const int32_t* counts, const int32_t* offsets, int S, int E, int d, int d_ff,
-                               uint8_t* hq, float* hs, int32_t* status) {
+                               uint8_t* hq, float* hs, int32_t* status, int act_rows) {
     if (S == 0) return cudaSuccess;
-    fp8::Args a{counts, offsets, E, d, d_ff, xq, xs, gather, Wg_s, Wu_s, hq, hs, nullptr, status};
+    fp8::Args a{counts, offsets, E, d, d_ff, xq, xs, gather, Wg_s, Wu_s, hq, hs, nullptr, status, S,
+                gather ? act_rows : S};
     if (fp8_rows(S, E) == 16) return fp8::run<true, 16>(c, S, Wg, Wu, a);
     return fp8::run<true, 32>(c, S, Wg, Wu, a);
 }
@@ -670,7 +687,7 @@ cudaError_t launch_down_fp8(const Ctx& c, const uint8_t* hq, const float* hs, co
                             int32_t* status) {
     if (S == 0) return cudaSuccess;
     fp8::Args a{counts, offsets, E, d_ff, d, hq, hs, nullptr, Wd_s, nullptr, nullptr, nullptr,
-                static_cast<uint16_t*>(y), status};
+                static_cast<uint16_t*>(y), status, S, S};
     // two 128-row weight blocks per tile where d allows: each promotion pass then covers 32 KB of
     // weights instead of 16 (the pass, not the MMAs or the loads, paces the 128-row tile)
     const bool wide = d % 256 == 0;

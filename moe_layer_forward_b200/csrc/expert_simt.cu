@@ -23,18 +23,25 @@ __global__ void __launch_bounds__(256) simt_grouped_kernel(const float* __restri
                                                            const float* __restrict__ W2,
                                                            const int32_t* __restrict__ counts,
                                                            const int32_t* __restrict__ offsets, int E, int K, int N,
-                                                           float* __restrict__ C) {
+                                                           float* __restrict__ C, int S, int32_t* status) {
     __shared__ int rb_start[kMaxExperts + 1];
+    __shared__ int cnt_s[kMaxExperts], off_s[kMaxExperts];
     __shared__ float As[SK][SR + 1];
     __shared__ float B1[SK][SC + 1];
     __shared__ float B2[SWIGLU ? SK : 1][SC + 1];
     pdl_wait();
     pdl_trigger();
     if (threadIdx.x == 0) {
+        // segments that do not fit the S-row buffers are clamped into them and flagged (by block 0)
         int run = 0;
         for (int e = 0; e < E; ++e) {
+            int o, n;
+            if (!clamp_segment(offsets[e], counts[e], S, o, n) && blockIdx.x == 0 && blockIdx.y == 0)
+                set_status(status, DEV_BAD_COUNT);
+            cnt_s[e] = n;
+            off_s[e] = o;
             rb_start[e] = run;
-            run += (counts[e] + SR - 1) / SR;
+            run += (n + SR - 1) / SR;
         }
         rb_start[E] = run;
     }
@@ -48,8 +55,8 @@ __global__ void __launch_bounds__(256) simt_grouped_kernel(const float* __restri
     }
     const int e = lo;
     const int rb = rbg - rb_start[e];
-    const int64_t row0 = (int64_t)offsets[e] + (int64_t)rb * SR;
-    const int rows = min(SR, counts[e] - rb * SR);
+    const int64_t row0 = (int64_t)off_s[e] + (int64_t)rb * SR;
+    const int rows = min(SR, cnt_s[e] - rb * SR);
     const int col0 = blockIdx.y * SC;
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
     float g[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, u[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
@@ -104,17 +111,17 @@ static dim3 simt_grid(int S, int E, int N) {
 }
 
 cudaError_t launch_gate_up_f32(const Ctx& c, const float* xp, const float* Wg, const float* Wu, const int32_t* counts,
-                               const int32_t* offsets, int S, int E, int d, int d_ff, float* h) {
+                               const int32_t* offsets, int S, int E, int d, int d_ff, float* h, int32_t* status) {
     if (S == 0) return cudaSuccess;
     return launch(simt_grouped_kernel<true>, simt_grid(S, E, d_ff), dim3(256), 0, c, xp, Wg, Wu, counts, offsets, E,
-                  d, d_ff, h);
+                  d, d_ff, h, S, status);
 }
 
 cudaError_t launch_down_f32(const Ctx& c, const float* h, const float* Wd, const int32_t* counts,
-                            const int32_t* offsets, int S, int E, int d, int d_ff, float* y) {
+                            const int32_t* offsets, int S, int E, int d, int d_ff, float* y, int32_t* status) {
     if (S == 0) return cudaSuccess;
     return launch(simt_grouped_kernel<false>, simt_grid(S, E, d), dim3(256), 0, c, h, Wd, (const float*)nullptr,
-                  counts, offsets, E, d_ff, d, y);
+                  counts, offsets, E, d_ff, d, y, S, status);
 }
 
 }  // namespace moe

@@ -118,6 +118,10 @@ struct Args {
     // Masked layout (cap > 0): expert e's rows are rows [e*cap, e*cap + counts[e]) of fixed
     // per-expert buffers, offsets is unused, and a count outside [0, cap] is clamped and flagged.
     int cap;
+    // rows of the expert-contiguous buffers (the output's rows); a segment that does not fit is
+    // clamped into it and flagged
+    int S;
+    int act_rows;  // rows of act when gather is set
 };
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
@@ -191,8 +195,10 @@ __global__ void __launch_bounds__(threads_of<SWAP>(), 1)
             aux.cnt[e] = n < 0 ? 0 : (n > p.cap ? p.cap : n);
             aux.off[e] = e * p.cap;
         } else {
-            aux.cnt[e] = p.counts[e];
-            aux.off[e] = p.offsets[e];
+            int o, n;
+            if (!clamp_segment(p.offsets[e], p.counts[e], p.S, o, n)) set_status(p.status, DEV_BAD_COUNT);
+            aux.cnt[e] = n;
+            aux.off[e] = o;
         }
     }
     __syncthreads();
@@ -373,7 +379,12 @@ __global__ void __launch_bounds__(threads_of<SWAP>(), 1)
 #pragma unroll
                     for (int i = 0; i < RPL; ++i) {
                         const int r = r0 + 4 * i;
-                        tok[i] = r < rows ? p.gather[base + r] : 0;
+                        int tk = r < rows ? p.gather[base + r] : 0;
+                        if (tk < 0 || tk >= p.act_rows) {  // a bad map entry reads row 0 instead and is flagged
+                            if (c == 0) set_status(p.status, DEV_BAD_COUNT);
+                            tk = 0;
+                        }
+                        tok[i] = tk;
                     }
                     cur = tile;
                 }
@@ -570,7 +581,7 @@ cudaError_t launch_gate_up_bf16(const Ctx& c, const void* xp, const void* Wg, co
     if (cap == 0 && use_pair_gemm(Ss, E, 256))
         return launch_gate_up_bf16_pair(c, xp, Wg, Wu, counts, offsets, S, E, d, d_ff, h, status);
     tc::Args a{counts, offsets, E, d, d_ff, static_cast<uint16_t*>(h), (int64_t)d_ff, status, gather,
-               static_cast<const uint16_t*>(xp), cap};
+               static_cast<const uint16_t*>(xp), cap, S, gather ? act_rows : 0};
     const int ar = gather ? act_rows : -1;
     switch (tc::pick_swap_rows(Ss, E)) {
         case 16: return tc::run<true, true, 16, 128>(c, xp, S, Wg, Wu, a, ar);
@@ -587,7 +598,7 @@ cudaError_t launch_down_bf16(const Ctx& c, const void* h, const void* Wd, const 
     const int Ss = S_sel > 0 ? S_sel : S;
     if (cap == 0 && use_pair_gemm(Ss, E, d))
         return launch_down_bf16_pair(c, h, Wd, counts, offsets, S, E, d, d_ff, y, status);
-    tc::Args a{counts, offsets, E, d_ff, d, static_cast<uint16_t*>(y), (int64_t)d, status, nullptr, nullptr, cap};
+    tc::Args a{counts, offsets, E, d_ff, d, static_cast<uint16_t*>(y), (int64_t)d, status, nullptr, nullptr, cap, S, 0};
     const int ra = tc::pick_rows(Ss, E);
     if (d % 256 == 0) {
         switch (ra) {

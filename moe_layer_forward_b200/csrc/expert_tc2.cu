@@ -69,6 +69,7 @@ struct Args2 {
     uint16_t* out;
     int64_t ldo;
     int32_t* status;
+    int S;  // rows of the expert-contiguous buffers; a segment that does not fit is clamped and flagged
 };
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -171,8 +172,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     pdl_wait();
     const int E = p.E;
     for (int e = threadIdx.x; e < E; e += kThreads) {
-        aux.cnt[e] = p.counts[e];
-        aux.off[e] = p.offsets[e];
+        int o, n;
+        if (!clamp_segment(p.offsets[e], p.counts[e], p.S, o, n) && leader) set_status(p.status, DEV_BAD_COUNT);
+        aux.cnt[e] = n;
+        aux.off[e] = o;
     }
     __syncthreads();
     const int ncb = p.n_out / WCOLS;
@@ -421,14 +424,14 @@ cudaError_t launch_gate_up_bf16_pair(const Ctx& c, const void* xp, const void* W
                                      const int32_t* counts, const int32_t* offsets, int S, int E, int d, int d_ff,
                                      void* h, int32_t* status) {
     if (S == 0) return cudaSuccess;
-    tc2::Args2 a{counts, offsets, E, d, d_ff, static_cast<uint16_t*>(h), (int64_t)d_ff, status};
+    tc2::Args2 a{counts, offsets, E, d, d_ff, static_cast<uint16_t*>(h), (int64_t)d_ff, status, S};
     return tc2::run2<true>(c, xp, S, Wg, Wu, a);
 }
 
 cudaError_t launch_down_bf16_pair(const Ctx& c, const void* h, const void* Wd, const int32_t* counts,
                                   const int32_t* offsets, int S, int E, int d, int d_ff, void* y, int32_t* status) {
     if (S == 0) return cudaSuccess;
-    tc2::Args2 a{counts, offsets, E, d_ff, d, static_cast<uint16_t*>(y), (int64_t)d, status};
+    tc2::Args2 a{counts, offsets, E, d_ff, d, static_cast<uint16_t*>(y), (int64_t)d, status, S};
     return tc2::run2<false>(c, h, S, Wd, nullptr, a);
 }
 

@@ -74,13 +74,13 @@ cudaError_t launch_permute(const Ctx& c, const void* v, int v_dt, const int32_t*
 // table [N][E]: rows every rank routes to every expert; recv / y: device arrays of N peer pointers
 cudaError_t launch_ep_dispatch(const Ctx& c, const void* v, int v_dt, const int32_t* idx, const int32_t* token_slot,
                                const int32_t* offsets, const int32_t* table, int rank, int N, int E, int T, int d,
-                               int k, void* const* recv, int32_t* status);
+                               int k, void* const* recv, int64_t recv_rows, int32_t* status);
 cudaError_t launch_ep_layout(const Ctx& c, const int32_t* table, int rank, int N, int E, int32_t* counts_loc,
                              int32_t* offsets_loc);
 cudaError_t launch_ep_combine(const Ctx& c, const void* const* y, int y_dt, const int32_t* idx,
                               const int32_t* token_slot, const int32_t* offsets, const int32_t* table, int rank, int N,
                               int E, const float* w, const void* res, int r_dt, int T, int d, int k, void* out,
-                              int out_dt, int32_t* status);
+                              int out_dt, int64_t recv_rows, int32_t* status);
 
 // ---- step 4: expert MLP (expert_tc.cu: bf16 tensor cores; expert_simt.cu: fp32)
 // gate/up: xp holds the S permuted rows; or, with gather, xp holds act_rows rows and slot i
@@ -111,14 +111,14 @@ cudaError_t launch_rmsnorm_quant(const Ctx& c, const void* x, int x_dt, const fl
 cudaError_t launch_gate_up_fp8(const Ctx& c, const uint8_t* xq, const float* xs, const int32_t* gather,
                                const uint8_t* Wg, const float* Wg_s, const uint8_t* Wu, const float* Wu_s,
                                const int32_t* counts, const int32_t* offsets, int S, int E, int d, int d_ff,
-                               uint8_t* hq, float* hs, int32_t* status);
+                               uint8_t* hq, float* hs, int32_t* status, int act_rows);
 cudaError_t launch_down_fp8(const Ctx& c, const uint8_t* hq, const float* hs, const uint8_t* Wd, const float* Wd_s,
                             const int32_t* counts, const int32_t* offsets, int S, int E, int d, int d_ff, void* y,
                             int32_t* status);
 cudaError_t launch_gate_up_f32(const Ctx& c, const float* xp, const float* Wg, const float* Wu, const int32_t* counts,
-                               const int32_t* offsets, int S, int E, int d, int d_ff, float* h);
+                               const int32_t* offsets, int S, int E, int d, int d_ff, float* h, int32_t* status);
 cudaError_t launch_down_f32(const Ctx& c, const float* h, const float* Wd, const int32_t* counts,
-                            const int32_t* offsets, int S, int E, int d, int d_ff, float* y);
+                            const int32_t* offsets, int S, int E, int d, int d_ff, float* y, int32_t* status);
 
 // ---- step 5: weighted un-permute + residual (combine.cu)
 cudaError_t launch_combine(const Ctx& c, const void* y, int y_dt, const int32_t* token_slot, const float* w,

@@ -26,19 +26,20 @@ constexpr size_t kStaticWords = (size_t)(kStaticMaxTokens / moe::kPermuteChunk) 
 static __device__ __align__(256) int32_t g_permute_scratch[kStaticWords];
 
 constexpr int kMaxDev = 64;
-std::once_flag g_once[kMaxDev];
+std::mutex g_lookup_mu;
 int32_t* g_scratch_ptr[kMaxDev] = {};
-cudaError_t g_scratch_err[kMaxDev] = {};
 
 // In host code g_permute_scratch names a host-side stand-in, not device memory,
-// so its device address is looked up once per device (with that device current).
+// so its device address is looked up per device (with that device current).
+// Only a successful lookup is kept: a call that failed (for example one made
+// during a stream capture) leaves the next call free to try again.
 int32_t* scratch_for(int dev) {
-    std::call_once(g_once[dev], [dev] {
+    std::lock_guard<std::mutex> lock(g_lookup_mu);
+    if (!g_scratch_ptr[dev]) {
         void* p = nullptr;
-        g_scratch_err[dev] = cudaGetSymbolAddress(&p, g_permute_scratch);
-        if (g_scratch_err[dev] == cudaSuccess) g_scratch_ptr[dev] = static_cast<int32_t*>(p);
+        if (cudaGetSymbolAddress(&p, g_permute_scratch) == cudaSuccess) g_scratch_ptr[dev] = static_cast<int32_t*>(p);
         else cudaGetLastError();
-    });
+    }
     return g_scratch_ptr[dev];
 }
 

@@ -118,7 +118,7 @@ class CudaP2POps(CudaOps):
         return counts, offsets, token_slot
 
     def dispatch(self, v, idx, token_slot, offsets, table, rank, peers: Peers):
-        self.m.moe_ep_dispatch(v, idx, token_slot, offsets, table, rank, peers.recv_ptrs)
+        self.m.moe_ep_dispatch(v, idx, token_slot, offsets, table, rank, peers.recv_ptrs, peers.rows)
 
     def layout(self, table, rank):
         N, E = table.shape
@@ -139,7 +139,7 @@ class CudaP2POps(CudaOps):
         out = torch.empty(residual.shape, dtype=out_dtype, device=residual.device)
         if residual.shape[0] > 0:
             self.m.moe_ep_combine(peers.y_ptrs, peers.y.dtype, idx, token_slot, offsets, table, rank, w, residual,
-                                  out)
+                                  out, peers.rows)
         return out
 
 
@@ -168,26 +168,39 @@ def _barrier(group, device):
 
 
 def ep_p2p_forward(x, gamma, W_r, b, W_gate_local, W_up_local, W_down_local, E: int, peers: Peers, T_max: int,
-                   top_k: int = 8, eps: float = 1e-5, group=None, ops=None, out_dtype=None):
+                   top_k: int = 8, eps: float = 1e-5, group=None, ops=None, out_dtype=None, agree_checks=True):
     """out = x + MoE(RMSNorm(x)) for this rank's tokens (one process per rank; collectives inside).
 
     W_*_local hold experts [rank E/N, (rank+1) E/N); peers holds buffers of at least
     capacity_rows(T_max, N, top_k, E) rows on every rank.  Returns (out, EPStats); the stats' rows_received
-    is a one-element device tensor (reading it is the only host synchronisation).  The argument checks run
-    before the first collective: a rank that fails one raises at once, and the other ranks' next collective
-    ends with the process group's timeout error."""
+    is a one-element device tensor.
+
+    With agree_checks (the default) the ranks first combine their argument checks in one all-reduce (MIN of
+    a pass flag) and read it on the host: if any rank fails a check, every rank raises ValueError together
+    and none is left waiting in a collective that a failed rank never joins.  That read is the step's one
+    host synchronisation; a caller that has validated its arguments once (e.g. before capturing the step in
+    a CUDA graph) passes agree_checks=False, and then a rank that fails a check raises alone while the
+    others' next collective ends with the process group's timeout error."""
     ops = ops or CudaP2POps()
     N = dist.get_world_size(group)
     rank = dist.get_rank(group)
+    problem = None
     if E % N != 0:
-        raise ValueError(f"{E} experts do not split over {N} ranks")
+        problem = f"{E} experts do not split over {N} ranks"
+    elif W_gate_local.shape[0] != E // N:
+        problem = f"rank {rank} holds {W_gate_local.shape[0]} experts, expected {E // N}"
+    elif x.shape[0] > T_max:
+        problem = f"rank {rank} has {x.shape[0]} tokens, more than T_max = {T_max}"
+    elif peers.rows < capacity_rows(T_max, N, top_k, E):
+        problem = f"peer buffers hold {peers.rows} rows, {capacity_rows(T_max, N, top_k, E)} needed"
+    if agree_checks:
+        ok = torch.tensor([0 if problem else 1], dtype=torch.int32, device=x.device)
+        dist.all_reduce(ok, op=dist.ReduceOp.MIN, group=group)
+        if problem is None and int(ok.item()) == 0:
+            problem = "another rank failed its argument checks (T_max, buffer rows or expert split)"
+    if problem is not None:
+        raise ValueError(problem)
     E_loc = E // N
-    if W_gate_local.shape[0] != E_loc:
-        raise ValueError(f"rank {rank} holds {W_gate_local.shape[0]} experts, expected {E_loc}")
-    if x.shape[0] > T_max:
-        raise ValueError(f"rank {rank} has {x.shape[0]} tokens, more than T_max = {T_max}")
-    if peers.rows < capacity_rows(T_max, N, top_k, E):
-        raise ValueError(f"peer buffers hold {peers.rows} rows, {capacity_rows(T_max, N, top_k, E)} needed")
     dev = x.device
     rt = _route(ops, x, gamma, W_r, b, E, top_k, eps, W_gate_local.dtype)
 

@@ -49,3 +49,18 @@ def check_routing(oracle_mod, logits, b, idx, w, k, ref_idx=None, ref_margin=Non
                 for a, c in zip(ri[t].tolist(), gi[t].tolist()):
                     assert abs(sc[a] - sc[c]) < NEAR_TIE, f"token {t}: pick order differs beyond a near-tie"
     return set_differs
+
+
+def oracle_fp8_weights(oracle_mod, W: torch.Tensor, device):
+    """Block-FP8 codes and scales of an expert weight tensor [E][n][k], quantised by the CPU oracle (so no
+    GPU value feeds the reference) and uploaded to `device` for the layer under test.  The experts are
+    quantised in parallel threads (the oracle's C calls release the GIL)."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    E, n, k = W.shape
+    W = W.detach().cpu().contiguous()
+    with ThreadPoolExecutor(max_workers=16) as ex:
+        parts = list(ex.map(lambda e: oracle_mod.quantize_blocks(W[e], 128), range(E)))
+    q = torch.stack([p[0] for p in parts])
+    s = torch.stack([p[1] for p in parts])
+    return q.to(device), s.to(device)

@@ -52,7 +52,7 @@ def test_status_strings_and_version(lib):
     texts = [lib.moe_status_string(s).decode() for s in range(6)]
     assert texts[0] == "ok" and len(set(texts)) == 6
     assert lib.moe_status_string(99).decode() == "unknown status"
-    assert lib.moe_abi_version() == 1
+    assert lib.moe_abi_version() == 2
 
 
 def test_launch_counter_counts_no_rejected_call(lib):
@@ -168,24 +168,28 @@ def test_peer_memory_and_sized_entries_reject_bad_arguments_on_host(lib):
     assert sz(_p(), _p(), _p(), _p(), 1, _p(), _p(), 64, 32, 8, 96, 256, _p(), _p(), NULL, NULL) == UNSUPPORTED
     assert sz(_p(), _p(), _p(), _p(), 1, NULL, _p(), 64, 32, 8, 128, 256, _p(), _p(), NULL, NULL) == INVALID
     dsp = lib.moe_ep_dispatch
-    dsp.argtypes = [V, ctypes.c_int, V, V, V, V, i32, i32, i32, i32, i32, i32, V, V, V]
-    assert dsp(_p(), 1, _p(), _p(), _p(), _p(), 0, 3, 16, 4, 64, 8, _p(), NULL, NULL) == UNSUPPORTED  # E % N
-    assert dsp(_p(), 1, _p(), _p(), _p(), _p(), 2, 2, 16, 4, 64, 8, _p(), NULL, NULL) == INVALID  # rank < N
-    assert dsp(_p(), 1, _p(), _p(), _p(), NULL, 0, 2, 16, 4, 64, 8, _p(), NULL, NULL) == INVALID  # table
-    assert dsp(_p(), 1, _p(), _p(), _p(), _p(), 0, 2, 16, 4, 60, 8, _p(), NULL, NULL) == UNSUPPORTED  # d % 8
-    assert dsp(_p(), 1, _p(), _p(), _p(), _p(), 0, 2, 16, 4, 64, 8, NULL, NULL, NULL) == INVALID  # recv_bufs
-    assert dsp(_p(), 1, _p(), _p(), _p(), _p(), 0, 2, 16, 0, 64, 8, _p(), NULL, NULL) == OK  # no tokens
+    i64 = ctypes.c_int64
+    dsp.argtypes = [V, ctypes.c_int, V, V, V, V, i32, i32, i32, i32, i32, i32, V, i64, V, V]
+    assert dsp(_p(), 1, _p(), _p(), _p(), _p(), 0, 3, 16, 4, 64, 8, _p(), 64, NULL, NULL) == UNSUPPORTED  # E % N
+    assert dsp(_p(), 1, _p(), _p(), _p(), _p(), 2, 2, 16, 4, 64, 8, _p(), 64, NULL, NULL) == INVALID  # rank < N
+    assert dsp(_p(), 1, _p(), _p(), _p(), NULL, 0, 2, 16, 4, 64, 8, _p(), 64, NULL, NULL) == INVALID  # table
+    assert dsp(_p(), 1, _p(), _p(), _p(), _p(), 0, 2, 16, 4, 60, 8, _p(), 64, NULL, NULL) == UNSUPPORTED  # d % 8
+    assert dsp(_p(), 1, _p(), _p(), _p(), _p(), 0, 2, 16, 4, 64, 8, NULL, 64, NULL, NULL) == INVALID  # recv_bufs
+    assert dsp(_p(), 1, _p(), _p(), _p(), _p(), 0, 2, 16, 4, 64, 8, _p(), -1, NULL, NULL) == INVALID  # recv_rows
+    assert dsp(_p(), 1, _p(), _p(), _p(), _p(), 0, 2, 16, 0, 64, 8, _p(), 64, NULL, NULL) == OK  # no tokens
     lay = lib.moe_ep_layout
     lay.argtypes = [V, i32, i32, i32, V, V, V]
     assert lay(NULL, 0, 2, 16, _p(), _p(), NULL) == INVALID
     assert lay(_p(), 0, 2, 16, NULL, _p(), NULL) == INVALID
     assert lay(_p(), 0, 5, 16, _p(), _p(), NULL) == UNSUPPORTED
     cmb = lib.moe_ep_combine
-    cmb.argtypes = [V, ctypes.c_int, V, V, V, V, i32, i32, i32, V, V, ctypes.c_int, i32, i32, i32, V, ctypes.c_int, V,
-                    V]
-    assert cmb(_p(), 1, _p(), _p(), _p(), _p(), 0, 2, 16, _p(), _p(), 1, 4, 64, 9, _p(), 1, NULL, NULL) == UNSUPPORTED
-    assert cmb(NULL, 1, _p(), _p(), _p(), _p(), 0, 2, 16, _p(), _p(), 1, 4, 64, 8, _p(), 1, NULL, NULL) == INVALID
-    assert cmb(_p(), 1, _p(), _p(), _p(), _p(), 0, 2, 16, _p(), _p(), 7, 4, 64, 8, _p(), 1, NULL, NULL) == INVALID
+    cmb.argtypes = [V, ctypes.c_int, V, V, V, V, i32, i32, i32, V, V, ctypes.c_int, i32, i32, i32, V, ctypes.c_int,
+                    i64, V, V]
+    assert cmb(_p(), 1, _p(), _p(), _p(), _p(), 0, 2, 16, _p(), _p(), 1, 4, 64, 9, _p(), 1, 64, NULL,
+               NULL) == UNSUPPORTED
+    assert cmb(NULL, 1, _p(), _p(), _p(), _p(), 0, 2, 16, _p(), _p(), 1, 4, 64, 8, _p(), 1, 64, NULL, NULL) == INVALID
+    assert cmb(_p(), 1, _p(), _p(), _p(), _p(), 0, 2, 16, _p(), _p(), 7, 4, 64, 8, _p(), 1, 64, NULL, NULL) == INVALID
+    assert cmb(_p(), 1, _p(), _p(), _p(), _p(), 0, 2, 16, _p(), _p(), 1, 4, 64, 8, _p(), 1, -1, NULL, NULL) == INVALID
 
 
 class Shape(ctypes.Structure):

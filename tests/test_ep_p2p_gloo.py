@@ -153,7 +153,7 @@ def test_capacity_covers_the_worst_case():
     assert ep_p2p.capacity_rows(10, 2, 8, 64) == 2 * 10 * 8
 
 
-def _failing_worker(rank, world, port, outdir, recv, y):
+def _failing_worker(rank, world, port, outdir, recv, y, agree):
     sys.path.insert(0, ROOT)
     sys.path.insert(0, os.path.join(ROOT, "tests"))
     import datetime
@@ -173,7 +173,7 @@ def _failing_worker(rank, world, port, outdir, recv, y):
     try:
         ep_p2p.ep_p2p_forward(x, I["gamma"], I["W_r"], I["b"], I["W_gate"][experts], I["W_up"][experts],
                               I["W_down"][experts], E=w.E, peers=ep_p2p.Peers(recv[rank], y[rank], recv, y),
-                              T_max=T_max, top_k=w.top_k, eps=w.eps, ops=_p2p_ops())
+                              T_max=T_max, top_k=w.top_k, eps=w.eps, ops=_p2p_ops(), agree_checks=agree)
     except ValueError as e:
         outcome = "ValueError: " + str(e)
     except RuntimeError as e:  # the collective that the failed rank never joins
@@ -181,7 +181,10 @@ def _failing_worker(rank, world, port, outdir, recv, y):
     torch.save({"outcome": outcome}, os.path.join(outdir, f"r{rank}.pt"))
 
 
-def test_a_rank_that_fails_its_checks_ends_the_others_collective_with_an_error():
+@pytest.mark.parametrize("agree", [True, False])
+def test_a_rank_that_fails_its_checks_stops_every_rank(agree):
+    # with the checks agreed in one all-reduce every rank raises ValueError together; without it the
+    # failing rank raises alone and the other's next collective ends with the group's timeout error
     from moe_layer_forward_b200 import ep_p2p
 
     world = 2
@@ -190,8 +193,11 @@ def test_a_rank_that_fails_its_checks_ends_the_others_collective_with_an_error()
     recv = [torch.zeros((rows, w.d), dtype=torch.float32).share_memory_() for _ in range(world)]
     y = [torch.zeros((rows, w.d), dtype=torch.float64).share_memory_() for _ in range(world)]
     with tempfile.TemporaryDirectory() as d:
-        mp.start_processes(_failing_worker, args=(world, _free_port(), d, recv, y), nprocs=world, join=True,
-                           start_method="spawn")
+        mp.start_processes(_failing_worker, args=(world, _free_port(), d, recv, y, agree), nprocs=world,
+                           join=True, start_method="spawn")
         r = [torch.load(os.path.join(d, f"r{k}.pt"))["outcome"] for k in range(world)]
     assert r[1].startswith("ValueError") and "T_max" in r[1]
-    assert r[0] == "RuntimeError"
+    if agree:
+        assert r[0].startswith("ValueError") and "another rank" in r[0]
+    else:
+        assert r[0] == "RuntimeError"

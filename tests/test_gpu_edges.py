@@ -7,7 +7,7 @@ import torch
 
 import oracle
 import synth
-from _layer_check import MAX_ABS, REL_L2, errors
+from _layer_check import MAX_ABS, REL_L2, errors, oracle_fp8_weights
 from test_gpu_parity import _check_layer
 
 pytestmark = pytest.mark.gpu
@@ -44,7 +44,7 @@ def test_forward_edge_shapes(moe, name):
 
 def _fp8_layer(moe, w, I):
     D = {n: cuda(t) for n, t in I.items()}
-    Wq = [moe.quantize_fp8_weights(D[n]) for n in ("W_gate", "W_up", "W_down")]
+    Wq = [oracle_fp8_weights(oracle, I[n], DEV) for n in ("W_gate", "W_up", "W_down")]
     out = torch.empty((w.T, w.d), dtype=w.out_dtype, device=DEV)
     idx = torch.empty((w.T, w.top_k), dtype=torch.int32, device=DEV)
     wt = torch.empty((w.T, w.top_k), dtype=torch.float32, device=DEV)

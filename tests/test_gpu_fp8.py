@@ -14,7 +14,7 @@ import torch
 
 import oracle
 import synth
-from _layer_check import MAX_ABS, REL_L2, errors
+from _layer_check import MAX_ABS, REL_L2, errors, oracle_fp8_weights
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -119,7 +119,7 @@ def test_fp8_forward_matches_oracle_composition(moe, name):
     w = synth.Workload(name, T, d, E, d_ff, x_dtype=xd, out_dtype=od, seed=820)
     I = synth.make_layer_inputs(w)
     D = {n: cuda(t) for n, t in I.items()}
-    Wq = [moe.quantize_fp8_weights(D[n]) for n in ("W_gate", "W_up", "W_down")]
+    Wq = [oracle_fp8_weights(oracle, I[n], DEV) for n in ("W_gate", "W_up", "W_down")]
     out = torch.empty((T, d), dtype=od, device=DEV)
     idx = torch.empty((T, 8), dtype=torch.int32, device=DEV)
     wt = torch.empty((T, 8), dtype=torch.float32, device=DEV)
@@ -153,7 +153,7 @@ def test_fp8_forward_full_decode_size_sampled(moe):
     w = synth.WORKLOADS["decode"]
     I = synth.make_layer_inputs(w)
     D = {n: cuda(t) for n, t in I.items()}
-    Wq = [moe.quantize_fp8_weights(D[n]) for n in ("W_gate", "W_up", "W_down")]
+    Wq = [oracle_fp8_weights(oracle, I[n], DEV) for n in ("W_gate", "W_up", "W_down")]
     out = torch.empty((w.T, w.d), dtype=w.out_dtype, device=DEV)
     idx = torch.empty((w.T, 8), dtype=torch.int32, device=DEV)
     wt = torch.empty((w.T, 8), dtype=torch.float32, device=DEV)

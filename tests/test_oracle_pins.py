@@ -408,3 +408,85 @@ def test_layer_bf16_inputs_are_read_exactly():
     a = oracle.moe_layer(I["x"], *args, I["W_gate"], I["W_up"], I["W_down"])
     c = oracle.moe_layer(I["x"].float(), *args, I["W_gate"].float(), I["W_up"].float(), I["W_down"].float())
     assert torch.equal(a["out"], c["out"])
+
+
+# --------------------------------------------------------------------------- grouped expert MLP (segments)
+def _labelled_experts(E, d):
+    """Experts whose MLP is y = (e + 1) * x exactly, for rows with x[0] == 1 and integer entries.
+
+    W_gate[e] maps every feature to 64 * x[0] = 64, where SiLU(64) = 64 exactly in fp64 (sigmoid(64)
+    rounds to 1); W_up[e] = (e + 1) * I; W_down[e] = I / 64 (a power of two).  So h = 64 (e + 1) x and
+    y = (e + 1) x, both exact: a row sent through the wrong expert, or left out, shows at once."""
+    Wg = torch.zeros((E, d, d))
+    Wg[:, :, 0] = 64.0
+    Wu = torch.stack([(e + 1) * torch.eye(d) for e in range(E)])
+    Wd = torch.stack([torch.eye(d) / 64.0 for _ in range(E)])
+    return Wg, Wu, Wd
+
+
+def _labelled_rows(S, d, seed):
+    x = synth.randint((S, d), seed, 1, -3, 3).double()
+    x[:, 0] = 1.0
+    return x.float()
+
+
+def _expected_grouped(x, counts, offsets, E):
+    """Row r of expert e's segment -> (e + 1) * x[r]; rows in no segment stay NaN (test-side restatement)."""
+    S, d = x.shape
+    h = torch.full((S, d), float("nan"), dtype=torch.float64)
+    y = torch.full((S, d), float("nan"), dtype=torch.float64)
+    for e in range(E):
+        lo, n = int(offsets[e]), int(counts[e])
+        y[lo:lo + n] = (e + 1) * x[lo:lo + n].double()
+        h[lo:lo + n] = 64.0 * (e + 1) * x[lo:lo + n].double()
+    return h, y
+
+
+@pytest.mark.parametrize("counts", [
+    [0, 3, 0, 1, 5, 0, 2],        # empty experts first, between and last-but-one; single-row segment
+    [4, 0, 0, 0, 0, 0, 1],        # the last expert owns the last row
+    [1, 1, 1, 1, 1, 1, 1, 1],     # every segment one row
+    [0, 0, 0, 9],                 # only the last expert has rows
+])
+def test_grouped_mlp_sends_each_segment_through_its_own_expert(counts):
+    E, d = len(counts), 8
+    c = torch.tensor(counts, dtype=torch.int32)
+    o = torch.zeros(E + 1, dtype=torch.int32)
+    o[1:] = torch.cumsum(c, 0)
+    x = _labelled_rows(int(c.sum()), d, 700 + E)
+    Wg, Wu, Wd = _labelled_experts(E, d)
+    h, y = oracle.grouped_mlp(x, c, o, Wg, Wu, Wd)
+    h_ref, y_ref = _expected_grouped(x, c, o, E)
+    assert torch.equal(y, y_ref) and torch.equal(h, h_ref)
+
+
+def test_grouped_mlp_leaves_rows_outside_every_segment_untouched():
+    # segments with gaps between them and rows past the last one: those rows keep their NaN fill
+    E, d, S = 4, 8, 20
+    c = torch.tensor([2, 0, 3, 4], dtype=torch.int32)
+    o = torch.tensor([1, 5, 6, 12, 16], dtype=torch.int32)  # rows 0, 3-5, 9-11 and 16-19 belong to no segment
+    x = _labelled_rows(S, d, 710)
+    Wg, Wu, Wd = _labelled_experts(E, d)
+    _, y = oracle.grouped_mlp(x, c, o, Wg, Wu, Wd)
+    _, y_ref = _expected_grouped(x, c, o, E)
+    covered = torch.zeros(S, dtype=torch.bool)
+    for e in range(E):
+        covered[int(o[e]):int(o[e]) + int(c[e])] = True
+    assert torch.isnan(y[~covered]).all()
+    assert torch.equal(y[covered], y_ref[covered])
+
+
+def test_grouped_mlp_over_the_permutation_reproduces_each_pick():
+    # real routing through oracle.permute and oracle.gather: the row that holds pick i of token t must
+    # come out as (idx[t][i] + 1) * v[t], the pick's own expert applied to its own token
+    T, E, k, d = 40, 6, 3, 8
+    idx = synth.distinct_topk(T, E, k, 720)
+    v = _labelled_rows(T, d, 721)
+    counts, offsets, slot_token, token_slot = oracle.permute(idx, E)
+    xp = oracle.gather(v, slot_token).float()
+    Wg, Wu, Wd = _labelled_experts(E, d)
+    _, y = oracle.grouped_mlp(xp, counts, offsets, Wg, Wu, Wd)
+    for t in range(T):
+        for i in range(k):
+            r = int(token_slot[t, i])
+            assert torch.equal(y[r], (int(idx[t, i]) + 1) * v[t].double())

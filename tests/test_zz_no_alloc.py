@@ -38,7 +38,8 @@ def _buffers(T, E, k, d, dtype):
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_static_scratch_permute_matches_workspace_permute_twice(moe, dtype):
     # two calls in a row with different sizes: the second must not see the first's leftovers
-    for (T, E, k, d, seed) in [(1000, 64, 8, 128, 1), (300, 256, 8, 64, 2)]:
+    # the last case is the documented maximum: 65536 tokens and 256 experts fill all 256 x 256 counters
+    for (T, E, k, d, seed) in [(1000, 64, 8, 128, 1), (300, 256, 8, 64, 2), (65536, 256, 8, 8, 3)]:
         idx = synth.distinct_topk(T, E, k, seed).to(DEV)
         v = synth.normal((T, d), seed, 1, dtype=dtype).to(DEV)
         ref = _buffers(T, E, k, d, dtype)
