@@ -378,6 +378,22 @@ moe_status_t moe_ep_combine(const void* const* y_bufs, moe_dtype_t y_dt, const i
  * made, e.g. to count the kernels of a timed loop.  Never fails. */
 uint64_t moe_kernel_launches(void);
 
+/*
+ * Limit of the bounded waits inside the tensor-core kernels (expert GEMMs,
+ * router logits), for every launch this process queues after the call; not
+ * part of any method on the pages.  Every wait of those kernels on another of
+ * their roles (a filled stage, a drained accumulator) gives up after
+ * limit_ns nanoseconds (0 restores the default, 2 s): the kernel then sets
+ * MOE_DEV_TIMEOUT in dev_status, stops its other roles, waits (bounded by a
+ * separate 2 s limit, never cut short) for the copies and MMAs it has already
+ * issued, frees its tensor memory and returns, so the context stays usable.
+ * inject_stall != 0 is for tests of that path only: each of those kernels
+ * then also waits once, before its first output tile, on a barrier that
+ * nothing completes, so the wait runs out and the unwinding above happens on
+ * valid data.  Process-wide; not synchronised with work already queued.
+ */
+void moe_set_wait_limit(uint64_t limit_ns, int32_t inject_stall);
+
 /* ABI version of this header (bumped on any incompatible change). */
 #define MOE_ABI_VERSION 2
 int32_t moe_abi_version(void);

@@ -77,6 +77,8 @@ _lib.moe_status_string.argtypes = [ctypes.c_int]
 _lib.moe_status_string.restype = ctypes.c_char_p
 _lib.moe_abi_version.restype = ctypes.c_int32
 _lib.moe_kernel_launches.restype = ctypes.c_uint64
+_lib.moe_set_wait_limit.argtypes = [ctypes.c_uint64, ctypes.c_int32]
+_lib.moe_set_wait_limit.restype = None
 
 
 class MoEError(RuntimeError):
@@ -120,6 +122,12 @@ def _ws(query, device) -> torch.Tensor:
 
 def abi_version() -> int:
     return int(_lib.moe_abi_version())
+
+
+def set_wait_limit(limit_ns: int = 0, inject_stall: bool = False) -> None:
+    """Limit (ns) of the tensor-core kernels' bounded waits for launches queued from now on (0: the default
+    2 s); inject_stall makes each of them wait once on a barrier nothing completes (failure-path tests)."""
+    _lib.moe_set_wait_limit(int(limit_ns), 1 if inject_stall else 0)
 
 
 def kernel_launches() -> int:

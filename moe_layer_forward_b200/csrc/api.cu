@@ -9,6 +9,8 @@
 
 namespace moe {
 std::atomic<uint64_t> g_kernel_launches{0};
+std::atomic<uint64_t> g_wait_limit_ns{0};
+std::atomic<int> g_inject_stall{0};
 }  // namespace moe
 
 using namespace moe;
@@ -125,6 +127,11 @@ const char* moe_status_string(moe_status_t s) {
 int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
 
 uint64_t moe_kernel_launches(void) { return moe::g_kernel_launches.load(std::memory_order_relaxed); }
+
+void moe_set_wait_limit(uint64_t limit_ns, int32_t inject_stall) {
+    moe::g_wait_limit_ns.store(limit_ns, std::memory_order_relaxed);
+    moe::g_inject_stall.store(inject_stall != 0, std::memory_order_relaxed);
+}
 
 moe_status_t moe_rmsnorm(const void* x, moe_dtype_t x_dt, const float* gamma, int32_t T, int32_t d, float eps,
                          void* v, moe_dtype_t v_dt, moe_stream_t stream) {

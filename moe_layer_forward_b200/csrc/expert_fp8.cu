@@ -263,6 +263,10 @@ struct Args {
     int32_t* status;
     int S;                  // rows of the expert-contiguous outputs; a segment that does not fit is clamped and flagged
     int act_rows;           // rows of act when gather is set
+    // bounded waits: the limit of one wait, and (failure-path tests only) an extra wait on a barrier
+    // that nothing completes, made by the epilogue warps before their first tile
+    uint64_t wait_ns = kTimeoutNs;
+    int stall = 0;
 };
 
 // input row of expert-contiguous slot `slot`: the slot itself, or its entry of the gather map (a map
@@ -284,6 +288,7 @@ struct Aux {
     uint64_t cempty[8];
     uint64_t drain;
     uint64_t redbar;  // the 4 epilogue warps' per-tile rendezvous on red
+    uint64_t never;   // completed by nothing: the injected stall waits on it
     uint32_t tmem_slot;
     int abort_flag;
     float red[2][4][32];  // by tile parity: a warp reaches tile j+2's rendezvous only after all read tile j's
@@ -317,6 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     Aux& aux = *reinterpret_cast<Aux*>(smem + STAGES * C::STAGE_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int* abort_flag = &aux.abort_flag;
+    const uint64_t wait_ns = p.wait_ns;
 
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -329,6 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(smem_u32(&aux.drain), 1);
         mbar_init(smem_u32(&aux.redbar), 4);
+        mbar_init(smem_u32(&aux.never), 1);
         aux.abort_flag = 0;
         fence_mbar_init();
         tma_prefetch(&tm_w1);
@@ -395,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             for (int kb = 0; kb < nk; ++kb) {
                 const uint32_t full = smem_u32(&aux.full[stage]);
-                if (!warp_wait(smem_u32(&aux.empty[stage]), phase ^ 1u, abort_flag)) {
+                if (!warp_wait(smem_u32(&aux.empty[stage]), phase ^ 1u, abort_flag, wait_ns)) {
                     give_up();
                     ok = false;
                     break;
@@ -416,8 +423,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok) break;
         }
-        for (int s = 0; s < STAGES; ++s)
-            if (used & (1u << s)) mbar_wait(smem_u32(&aux.full[s]), (last_parity >> s) & 1u, abort_flag);
+        {
+            const uint64_t dl = drain_deadline();
+            for (int s = 0; s < STAGES; ++s)
+                if (used & (1u << s)) mbar_drain(smem_u32(&aux.full[s]), (last_parity >> s) & 1u, dl);
+        }
     } else if (warp == 1) {
         // ================= MMA issuer
         int stage = 0;
@@ -430,8 +440,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t idesc = idesc_e4m3(128, (rows + 15) & ~15);
             for (int kb = 0; kb < nk; ++kb, ++q) {
                 const uint32_t c = q % C::NBUF, use = q / C::NBUF;
-                if (!warp_wait(smem_u32(&aux.full[stage]), phase, abort_flag) ||
-                    !warp_wait(smem_u32(&aux.cempty[c]), (use & 1u) ^ 1u, abort_flag)) {
+                if (!warp_wait(smem_u32(&aux.full[stage]), phase, abort_flag, wait_ns) ||
+                    !warp_wait(smem_u32(&aux.cempty[c]), (use & 1u) ^ 1u, abort_flag, wait_ns)) {
                     give_up();
                     ok = false;
                     break;
@@ -459,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (lane == 0) {
             tc_commit(smem_u32(&aux.drain));
-            mbar_wait(smem_u32(&aux.drain), 0, abort_flag);
+            mbar_drain(smem_u32(&aux.drain), 0, drain_deadline());
         }
         __syncwarp();
     } else if (warp >= 6) {
@@ -471,7 +481,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int g = gw;; g += 4) {
             const int ti = g / nk, kb = g - ti * nk;
             const int tile = blockIdx.x + ti * gridDim.x;
-            if (tile >= total || *abort_flag) break;
+            // (no abort check here: a stage the producer armed is always filled, so its drain completes)
+            if (tile >= total) break;
             if (tile != cur) {
                 int e, rb, cb;
                 decode_tile(aux, E, R, tile, e, rb, cb);
@@ -486,7 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const int stage = g % STAGES;
             const uint32_t use = (uint32_t)(g / STAGES);
-            if (!warp_wait(smem_u32(&aux.empty[stage]), (use & 1u) ^ 1u, abort_flag)) {
+            if (!warp_wait(smem_u32(&aux.empty[stage]), (use & 1u) ^ 1u, abort_flag, wait_ns)) {
                 give_up();
                 break;
             }
@@ -510,6 +521,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int f = 32 * qw + lane;  // weight row inside the tile's 128
         uint32_t q = 0, j = 0;
         bool ok = true;
+        if (p.stall && !warp_wait(smem_u32(&aux.never), 0, abort_flag, wait_ns)) {
+            give_up();
+            ok = false;
+        }
         for (int tile = blockIdx.x; tile < total && ok && !*abort_flag; tile += gridDim.x, ++j) {
             int e, rb, cb;
             decode_tile(aux, E, R, tile, e, rb, cb);
@@ -535,7 +550,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     sa_n = lane < rows ? __ldg(p.act_s + (int64_t)my_row * nk + kb + 1) : 0.f;
                 }
                 const uint32_t c = q % C::NBUF, use = q / C::NBUF;
-                if (!warp_wait(smem_u32(&aux.cfull[c]), use & 1u, abort_flag)) {
+                if (!warp_wait(smem_u32(&aux.cfull[c]), use & 1u, abort_flag, wait_ns)) {
                     give_up();
                     ok = false;
                     break;
@@ -570,7 +585,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&aux.redbar));
-                if (!warp_wait(smem_u32(&aux.redbar), j & 1u, abort_flag)) {
+                if (!warp_wait(smem_u32(&aux.redbar), j & 1u, abort_flag, wait_ns)) {
                     give_up();
                     break;
                 }
@@ -617,8 +632,9 @@ static bool encode_u8(CUtensorMap* tm, const void* base, uint64_t inner, uint64_
 }
 
 template <bool SWIGLU, int R, int NA = 2>
-static cudaError_t run(const Ctx& c, int S, const void* w1, const void* w2, const Args& a) {
+static cudaError_t run(const Ctx& c, int S, const void* w1, const void* w2, Args a) {
     using CF = Cfg<SWIGLU, R, NA>;
+    set_wait_args(a);
     auto kern = grouped_gemm_fp8_kernel<SWIGLU, R, NA>;
     static bool attr_done[64] = {};
     if (c.device < 0 || c.device >= 64) return cudaErrorInvalidDevice;

@@ -122,6 +122,10 @@ struct Args {
     // clamped into it and flagged
     int S;
     int act_rows;  // rows of act when gather is set
+    // bounded waits: the limit of one wait, and (failure-path tests only) an extra wait on a barrier
+    // that nothing completes, made by the epilogue warps before their first tile
+    uint64_t wait_ns = kTimeoutNs;
+    int stall = 0;
 };
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
@@ -135,6 +139,7 @@ struct Aux {  // lives after the stage ring in shared memory
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint64_t drain;
+    uint64_t never;  // completed by nothing: the injected stall waits on it
     uint32_t tmem_slot;
     int abort_flag;
     int tstart[kMaxExperts + 1];
@@ -166,6 +171,7 @@ __global__ void __launch_bounds__(threads_of<SWAP>(), 1)
     Aux& aux = *reinterpret_cast<Aux*>(smem + STAGES * C::STAGE_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int* abort_flag = &aux.abort_flag;
+    const uint64_t wait_ns = p.wait_ns;
 
     // ---- prologue (overlaps the previous kernel's tail under PDL)
     if (warp == 0 && lane == 0) {
@@ -178,6 +184,7 @@ __global__ void __launch_bounds__(threads_of<SWAP>(), 1)
             mbar_init(smem_u32(&aux.tempty[b]), 4);
         }
         mbar_init(smem_u32(&aux.drain), 1);
+        mbar_init(smem_u32(&aux.never), 1);
         aux.abort_flag = 0;
         fence_mbar_init();
         tma_prefetch(&tm_act);
@@ -247,7 +254,7 @@ __global__ void __launch_bounds__(threads_of<SWAP>(), 1)
             const int w_row = e * p.n_out + cb * COLS;
             for (int kb = 0; kb < nk; ++kb) {
                 const uint32_t full = smem_u32(&aux.full[stage]), empty = smem_u32(&aux.empty[stage]);
-                if (!warp_wait(empty, phase ^ 1u, abort_flag)) {
+                if (!warp_wait(empty, phase ^ 1u, abort_flag, wait_ns)) {
                     if (lane == 0) {
                         *abort_flag = 1;
                         set_status(p.status, DEV_TIMEOUT);
@@ -278,8 +285,11 @@ __global__ void __launch_bounds__(threads_of<SWAP>(), 1)
             }
         }
         // make sure no copy into this CTA's shared memory is still in flight
-        for (int s = 0; s < STAGES; ++s)
-            if (used & (1u << s)) mbar_wait(smem_u32(&aux.full[s]), (last_parity >> s) & 1u, abort_flag);
+        {
+            const uint64_t dl = drain_deadline();
+            for (int s = 0; s < STAGES; ++s)
+                if (used & (1u << s)) mbar_drain(smem_u32(&aux.full[s]), (last_parity >> s) & 1u, dl);
+        }
     } else if (warp == 1) {
         // ================= MMA issuer
         int stage = 0;
@@ -289,7 +299,7 @@ __global__ void __launch_bounds__(threads_of<SWAP>(), 1)
         for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x, ++j) {
             const int buf = j & 1;
             const uint32_t use = (uint32_t)(j >> 1);
-            if (!warp_wait(smem_u32(&aux.tempty[buf]), (use & 1u) ^ 1u, abort_flag)) {
+            if (!warp_wait(smem_u32(&aux.tempty[buf]), (use & 1u) ^ 1u, abort_flag, wait_ns)) {
                 if (lane == 0) {
                     *abort_flag = 1;
                     set_status(p.status, DEV_TIMEOUT);
@@ -309,7 +319,7 @@ __global__ void __launch_bounds__(threads_of<SWAP>(), 1)
             const uint32_t d_tmem = tmem_base + (uint32_t)(buf * C::ACC);
             bool ok = true;
             for (int kb = 0; kb < nk; ++kb) {
-                if (!warp_wait(smem_u32(&aux.full[stage]), phase, abort_flag)) {
+                if (!warp_wait(smem_u32(&aux.full[stage]), phase, abort_flag, wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -351,7 +361,7 @@ __global__ void __launch_bounds__(threads_of<SWAP>(), 1)
         // all MMAs of this thread complete before tensor memory is freed
         if (lane == 0) {
             tc_commit(smem_u32(&aux.drain));
-            mbar_wait(smem_u32(&aux.drain), 0, abort_flag);
+            mbar_drain(smem_u32(&aux.drain), 0, drain_deadline());
         }
         __syncwarp();
     } else if (SWAP && warp >= 6) {
@@ -370,7 +380,8 @@ __global__ void __launch_bounds__(threads_of<SWAP>(), 1)
             for (int g = gw;; g += 4) {
                 const int ti = g / nk, kb = g - ti * nk;
                 const int tile = blockIdx.x + ti * gridDim.x;
-                if (tile >= total || *abort_flag) break;
+                // (no abort check here: a stage the producer armed is always filled, so its drain completes)
+                if (tile >= total) break;
                 if (tile != cur) {
                     int e, rb, cb;
                     decode_tile(aux, E, R, tile, e, rb, cb);
@@ -390,7 +401,7 @@ __global__ void __launch_bounds__(threads_of<SWAP>(), 1)
                 }
                 const int stage = g % STAGES;
                 const uint32_t use = (uint32_t)(g / STAGES);
-                if (!warp_wait(smem_u32(&aux.empty[stage]), (use & 1u) ^ 1u, abort_flag)) {
+                if (!warp_wait(smem_u32(&aux.empty[stage]), (use & 1u) ^ 1u, abort_flag, wait_ns)) {
                     if (lane == 0) {
                         *abort_flag = 1;
                         set_status(p.status, DEV_TIMEOUT);
@@ -415,10 +426,14 @@ __global__ void __launch_bounds__(threads_of<SWAP>(), 1)
         // ================= epilogue (warps 2..5 -> TMEM lane quarters 2,3,0,1)
         const int q = warp & 3;
         int j = 0;
+        if (p.stall && !warp_wait(smem_u32(&aux.never), 0, abort_flag, wait_ns) && lane == 0) {
+            *abort_flag = 1;
+            set_status(p.status, DEV_TIMEOUT);
+        }
         for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x, ++j) {
             const int buf = j & 1;
             const uint32_t use = (uint32_t)(j >> 1);
-            if (!warp_wait(smem_u32(&aux.tfull[buf]), use & 1u, abort_flag)) {
+            if (!warp_wait(smem_u32(&aux.tfull[buf]), use & 1u, abort_flag, wait_ns)) {
                 if (lane == 0) {
                     *abort_flag = 1;
                     set_status(p.status, DEV_TIMEOUT);
@@ -517,8 +532,9 @@ static bool encode_2d(CUtensorMap* tm, const void* base, uint64_t inner, uint64_
 }
 
 template <bool SWAP, bool SWIGLU, int R, int COLS>
-static cudaError_t run(const Ctx& c, const void* act, int S, const void* w1, const void* w2, const Args& a,
+static cudaError_t run(const Ctx& c, const void* act, int S, const void* w1, const void* w2, Args a,
                        int act_rows = -1) {
+    set_wait_args(a);
     using C = Cfg<SWAP, SWIGLU, R, COLS>;
     auto kern = grouped_gemm_kernel<SWAP, SWIGLU, R, COLS>;
     static bool attr_done[64] = {};

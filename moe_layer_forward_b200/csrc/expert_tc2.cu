@@ -51,6 +51,7 @@ struct Aux2 {
     uint64_t tfull[2];       // each CTA: accumulator ready
     uint64_t tempty[2];      // leader CTA: both CTAs' epilogues drained the accumulator
     uint64_t drain;
+    uint64_t never;          // completed by nothing: the injected stall waits on it
     uint32_t tmem_slot;
     int abort_flag;
     int tstart[kMaxExperts + 1];
@@ -70,6 +71,10 @@ struct Args2 {
     int64_t ldo;
     int32_t* status;
     int S;  // rows of the expert-contiguous buffers; a segment that does not fit is clamped and flagged
+    // bounded waits: the limit of one wait, and (failure-path tests only) an extra wait on a barrier
+    // that nothing completes, made by the epilogue warps before their first tile
+    uint64_t wait_ns = kTimeoutNs;
+    int stall = 0;
 };
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -149,6 +154,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t rank = cluster_rank();
     const bool leader = rank == 0;
     volatile int* abort_flag = &aux.abort_flag;
+    const uint64_t wait_ns = p.wait_ns;
 
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -160,6 +166,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             mbar_init(smem_u32(&aux.tempty[b]), 8);
         }
         mbar_init(smem_u32(&aux.drain), 1);
+        mbar_init(smem_u32(&aux.never), 1);
         aux.abort_flag = 0;
         fence_mbar_init();
         tma_prefetch(&tm_act);
@@ -222,6 +229,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         uint32_t phase = 0;
         const int nk = p.K / BK;
         bool ok = true;
+        uint64_t last_issue = 0;
         for (int tile = cluster_id; tile < total && ok && !*abort_flag; tile += nclusters) {
             int e, rb, cb;
             decode_tile2(aux, E, tile, e, rb, cb);
@@ -229,7 +237,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int w_row = e * p.n_out + cb * WCOLS + (SWIGLU ? 0 : 128 * (int)rank);
             const CUtensorMap* tm_w = (SWIGLU && rank == 1) ? &tm_w2 : &tm_w1;
             for (int kb = 0; kb < nk; ++kb) {
-                if (!warp_wait(smem_u32(&aux.empty[stage]), phase ^ 1u, abort_flag)) {
+                if (!warp_wait(smem_u32(&aux.empty[stage]), phase ^ 1u, abort_flag, wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -239,6 +247,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     if (leader) mbar_expect_tx(smem_u32(&aux.full[stage]), 2 * STAGE_BYTES);
                     tma_load_2d_pair(a0, &tm_act, kb * BK, act_row, full_leader);
                     tma_load_2d_pair(a0 + STAGE_A, tm_w, kb * BK, w_row, full_leader);
+                    last_issue = globaltimer();
                 }
                 __syncwarp();
                 if (++stage == STAGES) {
@@ -248,6 +257,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
         }
         if (!ok) raise_abort();
+        // Unwinding: this CTA's loads complete on the leader's barrier, which the other CTA cannot wait
+        // on, so a producer that stopped early waits a fixed 200 us after its last load (a 32 KB copy
+        // from valid memory lands within microseconds) before the CTA may reach its teardown.
+        if (*abort_flag && lane == 0 && last_issue != 0)
+            while (globaltimer() < last_issue + 200000ull) {
+            }
+        __syncwarp();
     } else if (warp == 1) {
         // ================= MMA issuer (leader CTA only)
         if (leader) {
@@ -259,14 +275,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (int tile = cluster_id; tile < total && ok && !*abort_flag; tile += nclusters, ++j) {
                 const uint32_t idesc = idesc_bf16(256, 256);
                 const int buf = j & 1;
-                if (!warp_wait(smem_u32(&aux.tempty[buf]), ((uint32_t)(j >> 1) & 1u) ^ 1u, abort_flag)) {
+                if (!warp_wait(smem_u32(&aux.tempty[buf]), ((uint32_t)(j >> 1) & 1u) ^ 1u, abort_flag, wait_ns)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(buf * 256);
                 for (int kb = 0; kb < nk; ++kb) {
-                    if (!warp_wait(smem_u32(&aux.full[stage]), phase, abort_flag)) {
+                    if (!warp_wait(smem_u32(&aux.full[stage]), phase, abort_flag, wait_ns)) {
                         ok = false;
                         break;
                     }
@@ -292,7 +308,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (!ok) raise_abort();
             if (lane == 0) {
                 commit_pair_local(smem_u32(&aux.drain));
-                mbar_wait(smem_u32(&aux.drain), 0, abort_flag);
+                mbar_drain(smem_u32(&aux.drain), 0, drain_deadline());
             }
             __syncwarp();
         }
@@ -303,9 +319,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t tempty_leader1 = map_to_rank(smem_u32(&aux.tempty[1]), 0);
         int j = 0;
         bool ok = true;
+        if (p.stall && !warp_wait(smem_u32(&aux.never), 0, abort_flag, wait_ns)) ok = false;
         for (int tile = cluster_id; tile < total && ok && !*abort_flag; tile += nclusters, ++j) {
             const int buf = j & 1;
-            if (!warp_wait(smem_u32(&aux.tfull[buf]), (uint32_t)(j >> 1) & 1u, abort_flag)) {
+            if (!warp_wait(smem_u32(&aux.tfull[buf]), (uint32_t)(j >> 1) & 1u, abort_flag, wait_ns)) {
                 ok = false;
                 break;
             }
@@ -377,7 +394,8 @@ static bool encode(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t r
 }
 
 template <bool SWIGLU>
-static cudaError_t run2(const Ctx& c, const void* act, int S, const void* w1, const void* w2, const Args2& a) {
+static cudaError_t run2(const Ctx& c, const void* act, int S, const void* w1, const void* w2, Args2 a) {
+    set_wait_args(a);
     auto kern = grouped_gemm_2sm_kernel<SWIGLU>;
     static bool attr_done[64] = {};
     if (c.device < 0 || c.device >= 64) return cudaErrorInvalidDevice;

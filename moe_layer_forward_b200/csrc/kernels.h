@@ -13,6 +13,18 @@ namespace moe {
 // Kernels this library has enqueued in this process (successful launches only).
 extern std::atomic<uint64_t> g_kernel_launches;
 
+// Bounded waits of the tensor-core kernels, for launches queued from now on: the limit of one wait in
+// ns (0 = the kernels' default), and the failure-path test switch that makes each kernel's epilogue wait
+// once on a barrier that nothing completes (set through moe_set_wait_limit).
+extern std::atomic<uint64_t> g_wait_limit_ns;
+extern std::atomic<int> g_inject_stall;
+template <typename A>
+inline void set_wait_args(A& a) {
+    const uint64_t ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+    if (ns != 0) a.wait_ns = ns;
+    a.stall = g_inject_stall.load(std::memory_order_relaxed);
+}
+
 struct Ctx {
     cudaStream_t stream;
     int num_sms;

@@ -70,6 +70,7 @@ struct RAux {
     uint64_t cfull[2];   // chunk accumulator ready
     uint64_t cempty[2];  // chunk accumulator drained
     uint64_t drain;
+    uint64_t never;      // completed by nothing: the injected stall waits on it
     uint32_t tmem_slot;
     int abort_flag;
 };
@@ -84,6 +85,10 @@ struct RArgs {
     int ksplit;
     int slabs_per_split;
     int32_t* status;
+    // bounded waits: the limit of one wait, and (failure-path tests only) an extra wait on a barrier
+    // that nothing completes, made by the epilogue warps before their first tile
+    uint64_t wait_ns = kTimeoutNs;
+    int stall = 0;
 };
 
 __global__ void __launch_bounds__(256) router_wsplit_kernel(const float* __restrict__ W, int64_t n,
@@ -109,6 +114,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     RAux& aux = *reinterpret_cast<RAux*>(smem + STAGES * C::STAGE_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int* abort_flag = &aux.abort_flag;
+    const uint64_t wait_ns = p.wait_ns;
 
     if (warp == 0 && lane == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -120,6 +126,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(smem_u32(&aux.cempty[b]), 4);
         }
         mbar_init(smem_u32(&aux.drain), 1);
+        mbar_init(smem_u32(&aux.never), 1);
         aux.abort_flag = 0;
         fence_mbar_init();
         tma_prefetch(&tm_whi);
@@ -153,7 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int kb0 = split * p.slabs_per_split, kb1 = min(kslabs, kb0 + p.slabs_per_split);
             bool ok = true;
             for (int kb = kb0; kb < kb1; ++kb) {
-                if (!warp_wait(smem_u32(&aux.empty[stage]), phase ^ 1u, abort_flag)) {
+                if (!warp_wait(smem_u32(&aux.empty[stage]), phase ^ 1u, abort_flag, wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -176,8 +183,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
         }
-        for (int s = 0; s < STAGES; ++s)
-            if (used & (1u << s)) mbar_wait(smem_u32(&aux.full[s]), (last_parity >> s) & 1u, abort_flag);
+        {
+            const uint64_t dl = drain_deadline();
+            for (int s = 0; s < STAGES; ++s)
+                if (used & (1u << s)) mbar_drain(smem_u32(&aux.full[s]), (last_parity >> s) & 1u, dl);
+        }
     } else if (warp == 1) {
         // ================= MMA issuer: one chunk accumulator per kChunkSlabs stages, alternating
         int stage = 0;
@@ -190,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int kb0 = split * p.slabs_per_split, kb1 = min(kslabs, kb0 + p.slabs_per_split);
             for (int c0 = kb0; c0 < kb1 && ok; c0 += kChunkSlabs, ++g) {
                 const int buf = g & 1;
-                if (!warp_wait(smem_u32(&aux.cempty[buf]), ((uint32_t)(g >> 1) & 1u) ^ 1u, abort_flag)) {
+                if (!warp_wait(smem_u32(&aux.cempty[buf]), ((uint32_t)(g >> 1) & 1u) ^ 1u, abort_flag, wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -198,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t d_tmem = tmem_base + (uint32_t)((1 + buf) * NP);
                 const int c1 = min(kb1, c0 + kChunkSlabs);
                 for (int kb = c0; kb < c1; ++kb) {
-                    if (!warp_wait(smem_u32(&aux.full[stage]), phase, abort_flag)) {
+                    if (!warp_wait(smem_u32(&aux.full[stage]), phase, abort_flag, wait_ns)) {
                         ok = false;
                         break;
                     }
@@ -230,7 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) raise_abort();
         if (lane == 0) {
             tc_commit(smem_u32(&aux.drain));
-            mbar_wait(smem_u32(&aux.drain), 0, abort_flag);
+            mbar_drain(smem_u32(&aux.drain), 0, drain_deadline());
         }
         __syncwarp();
     } else if (warp < 2 + kProd) {
@@ -239,7 +249,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row = pt >> 1, half = pt & 1;
         int stage = 0;
         uint32_t phase = 0;
-        for (int u = blockIdx.x; u < units && !*abort_flag; u += gridDim.x) {
+        // no abort check in this loop: a stage whose slot was freed is always filled (so the TMA producer's
+        // drain of that stage completes); after an abort the next wait for a slot that is not free fails
+        for (int u = blockIdx.x; u < units; u += gridDim.x) {
             const int tile = u / per_tile, split = (u % per_tile) % p.ksplit;
             const int kb0 = split * p.slabs_per_split, kb1 = min(kslabs, kb0 + p.slabs_per_split);
             const int t = tile * BM + row;
@@ -273,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int i = 0; i < 16; ++i) v[i] = 0.f;
                 }
-                if (!warp_wait(smem_u32(&aux.empty[stage]), phase ^ 1u, abort_flag)) {
+                if (!warp_wait(smem_u32(&aux.empty[stage]), phase ^ 1u, abort_flag, wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -311,6 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q = warp & 3;
         int g = 0;
         bool ok = true;
+        if (p.stall && !warp_wait(smem_u32(&aux.never), 0, abort_flag, wait_ns)) ok = false;
         for (int u = blockIdx.x; u < units && ok && !*abort_flag; u += gridDim.x) {
             const int tile = u / per_tile, rem = u % per_tile, eblk = rem / p.ksplit, split = rem % p.ksplit;
             const int kb0 = split * p.slabs_per_split, kb1 = min(kslabs, kb0 + p.slabs_per_split);
@@ -321,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t lane_off = (uint32_t)(32 * q) << 16;
             for (int ci = 0; ci < nch; ++ci, ++g) {
                 const int buf = g & 1;
-                if (!warp_wait(smem_u32(&aux.cfull[buf]), (uint32_t)(g >> 1) & 1u, abort_flag)) {
+                if (!warp_wait(smem_u32(&aux.cfull[buf]), (uint32_t)(g >> 1) & 1u, abort_flag, wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -389,8 +402,9 @@ static bool encode_f32(CUtensorMap* tm, const void* base, uint64_t inner, uint64
 }
 
 template <int NP, bool NORM, int ADT>
-static cudaError_t run(const Ctx& c, const CUtensorMap& whi, const CUtensorMap& wlo, const RArgs& a, int units) {
+static cudaError_t run(const Ctx& c, const CUtensorMap& whi, const CUtensorMap& wlo, RArgs a, int units) {
     using C = RCfg<NP>;
+    set_wait_args(a);
     auto kern = router_tc_kernel<NP, NORM, ADT>;
     static bool attr_done[64] = {};
     if (c.device < 0 || c.device >= 64) return cudaErrorInvalidDevice;

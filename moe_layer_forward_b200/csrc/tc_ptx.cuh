@@ -10,7 +10,8 @@
 namespace moe {
 namespace tc {
 
-constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s per wait
+constexpr uint64_t kTimeoutNs = 2000000000ull;  // default limit of one wait: 2 s
+constexpr uint64_t kDrainNs = 2000000000ull;    // limit of all of one role's unwinding waits together
 
 // ----------------------------------------------------------------------------- PTX wrappers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -42,25 +43,39 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Wait for the phase of the given parity to complete.  Gives up after
-// kTimeoutNs, or early once another role has raised the abort flag.
-static __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+// Wait for the phase of the given parity to complete.  Gives up after limit_ns
+// (the kernel's wait limit, kTimeoutNs unless the caller set another), or early
+// once another role has raised the abort flag.
+static __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                              uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 127u) == 0u) {
             if (*abort_flag) return false;
-            if (globaltimer() - t0 > kTimeoutNs) return false;
+            if (globaltimer() - t0 > limit_ns) return false;
         }
     }
 }
 
 // Every lane of the warp waits; the result is the same for all lanes.
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-    const bool ok = mbar_wait(bar, parity, abort_flag);
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, uint64_t limit_ns) {
+    const bool ok = mbar_wait(bar, parity, abort_flag, limit_ns);
     return __all_sync(0xffffffffu, ok);
 }
+
+// A wait of the unwinding path: it ignores the abort flag and is bounded only
+// by `deadline` (a %globaltimer value shared by all of one role's drain waits),
+// so that a role waits for the copies and MMAs it issued before it frees
+// tensor memory or lets the CTA exit, whatever the other roles did.
+static __device__ __noinline__ bool mbar_drain(uint32_t bar, uint32_t parity, uint64_t deadline) {
+    for (uint32_t it = 0;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 127u) == 127u && globaltimer() > deadline) return false;
+    }
+}
+__device__ __forceinline__ uint64_t drain_deadline() { return globaltimer() + kDrainNs; }
 
 __device__ __forceinline__ void tma_prefetch(const CUtensorMap* tm) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tm)) : "memory");
