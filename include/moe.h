@@ -189,6 +189,19 @@ moe_status_t moe_expert_gate_up(const void* xp, const void* W_gate, const void* 
                                 int32_t d_ff, void* h, int32_t* dev_status, moe_stream_t stream);
 
 /*
+ * The gate/up GEMM core without its SwiGLU product, for testing the tensor-core
+ * arithmetic on its own (the pages have no such step):
+ *   gu[r][f]        = bf16(sum_j xp[r][j] W_gate[e][f][j])
+ *   gu[r][d_ff + f] = bf16(sum_j xp[r][j] W_up[e][f][j])
+ * for every row r of expert e's segment: the same kernels, tile forms and fp32
+ * accumulation as moe_expert_gate_up (bf16 only), with the epilogue storing
+ * the two sums instead of SiLU(g) * u.  gu [S][2 d_ff] bf16.
+ */
+moe_status_t moe_expert_gate_up_raw(const void* xp, const void* W_gate, const void* W_up, const int32_t* counts,
+                                    const int32_t* offsets, int32_t S, int32_t E, int32_t d, int32_t d_ff, void* gu,
+                                    int32_t* dev_status, moe_stream_t stream);
+
+/*
  * Step 4, second half — down projection [P1 §实际 MLP 计算策略, "· W_down"]:
  *   y[r][o] = sum_f h[r][f] W_down[e][o][f]   for rows r of expert e's segment.
  * h [S][d_ff], y [S][d] (dtype dt).  bf16 requires d % 128 == 0, d_ff % 64 == 0.

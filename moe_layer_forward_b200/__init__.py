@@ -52,6 +52,7 @@ _sig = {
     "moe_permute_static_ws": [_vp, _i32, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
     "moe_expert_gate_up": [_vp, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp],
     "moe_expert_down": [_vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp],
+    "moe_expert_gate_up_raw": [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp],
     "moe_grouped_swiglu": [_vp, _vp, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp],
     "moe_grouped_swiglu_masked": [_vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp],
     "moe_unpermute_combine": [_vp, _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _i32, _vp],
@@ -189,6 +190,15 @@ def moe_expert_gate_up(xp, W_gate, W_up, counts, offsets, h, dev_status=None) ->
     _check("moe_expert_gate_up", _lib.moe_expert_gate_up(_p(xp), _p(W_gate), _p(W_up), _dt(W_gate), _p(counts),
                                                          _p(offsets), S, E, d, d_ff, _p(h), _p(dev_status),
                                                          _stream(xp.device)))
+
+
+def moe_expert_gate_up_raw(xp, W_gate, W_up, counts, offsets, gu, dev_status=None) -> None:
+    """The gate/up GEMMs without the SwiGLU product: gu [S][2 d_ff] = [xp W_gate^T | xp W_up^T] per segment (bf16)."""
+    S, d = xp.shape
+    E, d_ff, _ = W_gate.shape
+    _check("moe_expert_gate_up_raw", _lib.moe_expert_gate_up_raw(_p(xp), _p(W_gate), _p(W_up), _p(counts),
+                                                                 _p(offsets), S, E, d, d_ff, _p(gu), _p(dev_status),
+                                                                 _stream(xp.device)))
 
 
 def moe_expert_down(h, W_down, counts, offsets, y, dev_status=None) -> None:

@@ -212,6 +212,21 @@ moe_status_t moe_expert_gate_up(const void* xp, const void* W_gate, const void* 
                                           static_cast<float*>(h), dev_status));
 }
 
+moe_status_t moe_expert_gate_up_raw(const void* xp, const void* W_gate, const void* W_up, const int32_t* counts,
+                                    const int32_t* offsets, int32_t S, int32_t E, int32_t d, int32_t d_ff, void* gu,
+                                    int32_t* dev_status, moe_stream_t stream) {
+    moe_status_t st = check_expert_shape(MOE_BF16, S, E, d, d_ff);
+    if (st != MOE_OK) return st;
+    if (S == 0) return MOE_OK;
+    if (!xp || !W_gate || !W_up || !counts || !offsets || !gu) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(xp) || !aligned16(W_gate) || !aligned16(W_up) || !aligned16(gu)) return MOE_ERR_INVALID_ARG;
+    Ctx c;
+    st = make_ctx(stream, c);
+    if (st != MOE_OK) return st;
+    return cuda_status(launch_gate_up_bf16(c, xp, W_gate, W_up, counts, offsets, S, E, d, d_ff, gu, dev_status,
+                                           nullptr, 0, 0, 0, true));
+}
+
 moe_status_t moe_expert_down(const void* h, const void* W_down, moe_dtype_t dt, const int32_t* counts,
                              const int32_t* offsets, int32_t S, int32_t E, int32_t d, int32_t d_ff, void* y,
                              int32_t* dev_status, moe_stream_t stream) {

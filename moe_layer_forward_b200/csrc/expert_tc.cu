@@ -126,6 +126,9 @@ struct Args {
     // that nothing completes, made by the epilogue warps before their first tile
     uint64_t wait_ns = kTimeoutNs;
     int stall = 0;
+    // GEMM-core test form of gate/up (SWIGLU only): g and u are stored apart as bf16, g in columns
+    // [0, n_out) and u in [n_out, 2 n_out) of an output with ldo = 2 n_out; no SwiGLU product
+    int raw = 0;
 };
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
@@ -461,6 +464,23 @@ __global__ void __launch_bounds__(threads_of<SWAP>(), 1)
                         tmem_ld32(tb + COLS + c, u);
                         tmem_wait_ld(g);
                         tmem_wait_ld(u);
+                        if (p.raw) {  // GEMM-core test form: g and u stored apart
+                            uint32_t pu[16];
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                pk[i] = pack_bf16x2(__uint_as_float(g[2 * i]), __uint_as_float(g[2 * i + 1]));
+                                pu[i] = pack_bf16x2(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1]));
+                            }
+                            if (valid) {
+#pragma unroll
+                                for (int v = 0; v < 4; ++v) {
+                                    st16(orow + c + 8 * v, make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]));
+                                    st16(orow + p.n_out + c + 8 * v,
+                                         make_uint4(pu[4 * v], pu[4 * v + 1], pu[4 * v + 2], pu[4 * v + 3]));
+                                }
+                            }
+                            continue;
+                        }
 #pragma unroll
                         for (int i = 0; i < 16; ++i)
                             pk[i] = pack_bf16x2(silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
@@ -489,6 +509,16 @@ __global__ void __launch_bounds__(threads_of<SWAP>(), 1)
                         tmem_ld(tb + R + c, u);
                         tmem_wait_ld(g);
                         tmem_wait_ld(u);
+                        if (p.raw) {  // GEMM-core test form: g and u stored apart
+#pragma unroll
+                            for (int i = 0; i < C::LDW; ++i)
+                                if (c + i < rows) {
+                                    ocol[(int64_t)(c + i) * p.ldo] = (uint16_t)f32_to_bf16_bits(__uint_as_float(g[i]));
+                                    ocol[(int64_t)(c + i) * p.ldo + p.n_out] =
+                                        (uint16_t)f32_to_bf16_bits(__uint_as_float(u[i]));
+                                }
+                            continue;
+                        }
 #pragma unroll
                         for (int i = 0; i < C::LDW; ++i)
                             if (c + i < rows)
@@ -590,14 +620,15 @@ bool gate_up_needs_permuted_rows(int S, int E) { return use_pair_gemm(S, E, 256)
 
 cudaError_t launch_gate_up_bf16(const Ctx& c, const void* xp, const void* Wg, const void* Wu, const int32_t* counts,
                                 const int32_t* offsets, int S, int E, int d, int d_ff, void* h, int32_t* status,
-                                const int32_t* gather, int act_rows, int cap, int S_sel) {
+                                const int32_t* gather, int act_rows, int cap, int S_sel, bool raw) {
     if (S == 0) return cudaSuccess;
     const int Ss = S_sel > 0 ? S_sel : S;  // rows the tile form is chosen for
     if (gather && (cap > 0 || gate_up_needs_permuted_rows(Ss, E))) return cudaErrorInvalidValue;
     if (cap == 0 && use_pair_gemm(Ss, E, 256))
-        return launch_gate_up_bf16_pair(c, xp, Wg, Wu, counts, offsets, S, E, d, d_ff, h, status);
-    tc::Args a{counts, offsets, E, d, d_ff, static_cast<uint16_t*>(h), (int64_t)d_ff, status, gather,
+        return launch_gate_up_bf16_pair(c, xp, Wg, Wu, counts, offsets, S, E, d, d_ff, h, status, raw);
+    tc::Args a{counts, offsets, E, d, d_ff, static_cast<uint16_t*>(h), (int64_t)d_ff * (raw ? 2 : 1), status, gather,
                static_cast<const uint16_t*>(xp), cap, S, gather ? act_rows : 0};
+    a.raw = raw ? 1 : 0;
     const int ar = gather ? act_rows : -1;
     switch (tc::pick_swap_rows(Ss, E)) {
         case 16: return tc::run<true, true, 16, 128>(c, xp, S, Wg, Wu, a, ar);

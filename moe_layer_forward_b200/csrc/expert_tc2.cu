@@ -75,6 +75,8 @@ struct Args2 {
     // that nothing completes, made by the epilogue warps before their first tile
     uint64_t wait_ns = kTimeoutNs;
     int stall = 0;
+    // GEMM-core test form of gate/up: g in columns [0, n_out), u in [n_out, 2 n_out), no SwiGLU product
+    int raw = 0;
 };
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -346,6 +348,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         tmem_ld32(tb_addr + 128 + c, u);
                         tmem_wait_ld(g);
                         tmem_wait_ld(u);
+                        if (p.raw) {  // GEMM-core test form: g and u stored apart
+                            uint32_t pu[16];
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                pk[i] = pack_bf16x2(__uint_as_float(g[2 * i]), __uint_as_float(g[2 * i + 1]));
+                                pu[i] = pack_bf16x2(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1]));
+                            }
+                            if (valid) {
+#pragma unroll
+                                for (int v = 0; v < 4; ++v) {
+                                    st16(orow + c + 8 * v, make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]));
+                                    st16(orow + p.n_out + c + 8 * v,
+                                         make_uint4(pu[4 * v], pu[4 * v + 1], pu[4 * v + 2], pu[4 * v + 3]));
+                                }
+                            }
+                            continue;
+                        }
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
                             const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
@@ -440,9 +459,10 @@ bool use_pair_gemm(int S, int E, int n_out) {
 
 cudaError_t launch_gate_up_bf16_pair(const Ctx& c, const void* xp, const void* Wg, const void* Wu,
                                      const int32_t* counts, const int32_t* offsets, int S, int E, int d, int d_ff,
-                                     void* h, int32_t* status) {
+                                     void* h, int32_t* status, bool raw) {
     if (S == 0) return cudaSuccess;
-    tc2::Args2 a{counts, offsets, E, d, d_ff, static_cast<uint16_t*>(h), (int64_t)d_ff, status, S};
+    tc2::Args2 a{counts, offsets, E, d, d_ff, static_cast<uint16_t*>(h), (int64_t)d_ff * (raw ? 2 : 1), status, S};
+    a.raw = raw ? 1 : 0;
     return tc2::run2<true>(c, xp, S, Wg, Wu, a);
 }
 

@@ -104,14 +104,15 @@ bool gate_up_needs_permuted_rows(int S, int E);
 // while the buffers hold S (the row count on the device decides the work either way).
 cudaError_t launch_gate_up_bf16(const Ctx& c, const void* xp, const void* Wg, const void* Wu, const int32_t* counts,
                                 const int32_t* offsets, int S, int E, int d, int d_ff, void* h, int32_t* status,
-                                const int32_t* gather = nullptr, int act_rows = 0, int cap = 0, int S_sel = 0);
+                                const int32_t* gather = nullptr, int act_rows = 0, int cap = 0, int S_sel = 0,
+                                bool raw = false);
 cudaError_t launch_down_bf16(const Ctx& c, const void* h, const void* Wd, const int32_t* counts, const int32_t* offsets,
                              int S, int E, int d, int d_ff, void* y, int32_t* status, int cap = 0, int S_sel = 0);
 // CTA-pair (cta_group::2) variants for experts with many rows each (expert_tc2.cu)
 bool use_pair_gemm(int S, int E, int n_out);
 cudaError_t launch_gate_up_bf16_pair(const Ctx& c, const void* xp, const void* Wg, const void* Wu,
                                      const int32_t* counts, const int32_t* offsets, int S, int E, int d, int d_ff,
-                                     void* h, int32_t* status);
+                                     void* h, int32_t* status, bool raw = false);
 cudaError_t launch_down_bf16_pair(const Ctx& c, const void* h, const void* Wd, const int32_t* counts,
                                   const int32_t* offsets, int S, int E, int d, int d_ff, void* y, int32_t* status);
 // Block-FP8 experts (expert_fp8.cu): E4M3 codes, fp32 scales per 128 x 128 weight block and per

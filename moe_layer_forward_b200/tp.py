@@ -56,3 +56,29 @@ def tp_forward(x, gamma, W_r, b, W_gate_slice, W_up_slice, W_down_slice, top_k: 
         return mine.to(out_dtype)
     dist.all_reduce(part, op=dist.ReduceOp.SUM, group=group)
     return part.to(out_dtype)
+
+
+def tp_partials_emulated(x, gamma, W_r, b, W_gate, W_up, W_down, N: int, top_k: int = 8, eps: float = 1e-5,
+                         ops=None):
+    """All N ranks of tp_forward in this process, on one device: the N fp32 partial outputs, before the
+    reduction.  Rank r runs the grouped MLP on the features [r F, (r+1) F) of every expert (F = d_ff / N,
+    a multiple of 128) and the weighted combine of its partial y, with the residual on rank 0 only; their
+    sum is the layer (the all-reduce), and rows [r T/N, (r+1) T/N) of the sum are rank r's block of the
+    reduce-scatter.  The routing is computed once: it is identical on every rank."""
+    ops = ops or CudaOps()
+    E, d_ff, _ = W_gate.shape
+    if d_ff % N != 0 or (d_ff // N) % 128 != 0:
+        raise ValueError(f"d_ff = {d_ff} does not split over {N} ranks in multiples of 128")
+    F = d_ff // N
+    v32 = ops.rmsnorm(x, gamma, eps, torch.float32)
+    vx = ops.rmsnorm(x, gamma, eps, W_gate.dtype)
+    idx, w = ops.router(v32, W_r, b, top_k)
+    counts, offsets, token_slot, xp = ops.permute(vx, idx, E)
+    parts = []
+    for r in range(N):
+        sl = slice(r * F, (r + 1) * F)
+        y_part = ops.grouped_swiglu(xp, W_gate[:, sl].contiguous(), W_up[:, sl].contiguous(),
+                                    W_down[:, :, sl].contiguous(), counts, offsets)
+        residual = x if r == 0 else torch.zeros_like(x)
+        parts.append(ops.combine(y_part, token_slot, w, residual, torch.float32))
+    return parts, idx, w

@@ -246,6 +246,31 @@ def test_expert_down_integer_inputs_bit_exact(moe, case):
     assert torch.equal(y.cpu().double(), ref)
 
 
+@pytest.mark.parametrize("case", list(COUNT_CASES))
+def test_expert_gate_up_core_integer_inputs_bit_exact(moe, case):
+    # the gate/up GEMMs with the SwiGLU product left out (moe_expert_gate_up_raw), every tile form: weights-as-M
+    # with 16/32/64 staged rows (ra16 .. ra128), rows-as-M one-CTA (ra128b, rows, rows256) and CTA pairs (pairs).
+    # Entries in {-1, 0, 1}: every fp32 partial sum is an integer and |g|, |u| <= d = 256, so both round to bf16
+    # exactly and must equal the oracle's linear map bit for bit
+    d, d_ff = 256, 256
+    counts, offsets = _segments(COUNT_CASES[case])
+    E, S = len(counts), int(counts.sum())
+    xp = synth.randint((S, d), 305, 1, -1, 1).to(torch.bfloat16)
+    Wg = synth.randint((E, d_ff, d), 305, 2, -1, 1).to(torch.bfloat16)
+    Wu = synth.randint((E, d_ff, d), 305, 3, -1, 1).to(torch.bfloat16)
+    gu = torch.full((S, 2 * d_ff), float("nan"), dtype=torch.bfloat16, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    moe.moe_expert_gate_up_raw(cuda(xp), cuda(Wg), cuda(Wu), cuda(counts), cuda(offsets), gu, dev_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    ref = torch.empty((S, 2 * d_ff), dtype=torch.float64)
+    for e in range(E):
+        for r in range(int(offsets[e]), int(offsets[e + 1])):
+            ref[r, :d_ff] = oracle.linear(xp[r].double(), Wg[e])
+            ref[r, d_ff:] = oracle.linear(xp[r].double(), Wu[e])
+    assert torch.equal(gu.cpu().double(), ref)
+
+
 @pytest.mark.parametrize("case", ["ra32", "rows"])
 def test_expert_mlp_f32(moe, case):
     d, d_ff = 64, 96
@@ -319,6 +344,30 @@ def _assert_rounding_bound(got, ref, x):
     assert ((got - ref).abs() <= bound).all(), ((got - ref).abs() - bound).max().item()
 
 
+def _oracle_layer(x, *args, **kw):
+    """oracle.moe_layer on the rows of x, in chunks on parallel threads (the C oracle releases the GIL; each
+    row is computed independently, so the result is the same as one call)."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+
+    n = x.shape[0]
+    workers = max(1, min(32, os.cpu_count() or 1, n // 4))
+    if workers == 1:
+        return oracle.moe_layer(x, *args, **kw)
+    bounds = [n * i // workers for i in range(workers + 1)]
+
+    def part(i):
+        lo, hi = bounds[i], bounds[i + 1]
+        kk = dict(kw)
+        if kk.get("force_idx") is not None:
+            kk["force_idx"], kk["force_w"] = kk["force_idx"][lo:hi], kk["force_w"][lo:hi]
+        return oracle.moe_layer(x[lo:hi], *args, **kk)
+
+    with ThreadPoolExecutor(max_workers=workers) as ex:
+        parts = list(ex.map(part, range(workers)))
+    return {k: torch.cat([p[k] for p in parts]) for k in parts[0]}
+
+
 def _check_layer(moe, w, I, tokens=None, result=None, spec_tolerance=True):
     out, idx, wt, logits = result if result is not None else _run_forward(moe, w, I)
     args = (I["gamma"], I["W_r"], I["b"], I["W_gate"], I["W_up"], I["W_down"])
@@ -326,7 +375,7 @@ def _check_layer(moe, w, I, tokens=None, result=None, spec_tolerance=True):
     check_routing(oracle, logits, I["b"], idx, wt, w.top_k)
     sel = torch.arange(w.T) if tokens is None else torch.tensor(tokens)
     x = I["x"][sel]
-    ref = oracle.moe_layer(x, *args, k=w.top_k, eps=w.eps)
+    ref = _oracle_layer(x, *args, k=w.top_k, eps=w.eps)
     z_err = (logits.cpu()[sel].double() - ref["z32"].double()).abs().max().item()
     assert z_err < 1e-4, z_err
     differs = check_routing(oracle, logits.cpu()[sel], I["b"], idx.cpu()[sel], wt.cpu()[sel], w.top_k,
@@ -343,7 +392,7 @@ def _check_layer(moe, w, I, tokens=None, result=None, spec_tolerance=True):
     moe_abs, moe_rel = errors(got[keep].double() - x[keep].double(), ref["out"][keep] - x[keep].double())
     assert moe_rel <= 2e-2, moe_rel
     # forced routing: the oracle follows the GPU's experts and weights, every token compared
-    forced = oracle.moe_layer(x, *args, k=w.top_k, eps=w.eps, force_idx=idx.cpu()[sel], force_w=wt.cpu()[sel])
+    forced = _oracle_layer(x, *args, k=w.top_k, eps=w.eps, force_idx=idx.cpu()[sel], force_w=wt.cpu()[sel])
     f_abs, f_rel = errors(got, forced["out"])
     if spec_tolerance:
         assert f_abs <= MAX_ABS and f_rel <= REL_L2, (f_abs, f_rel)
@@ -450,9 +499,28 @@ def test_forward_launch_count_is_reported_and_stable(moe):
 
 
 # --------------------------------------------------------------------------- full-size workloads (sampled)
-def _sample_tokens(T, n, seed):
-    raw = synth.raw_u64(n, seed, 99)
-    return sorted(set([0, T - 1] + [int(r % T) for r in raw]))[:n + 2]
+def _tile_covering_tokens(idx, E):
+    """Tokens whose rows include the first, a middle and the last row of every active expert's segment, so
+    that the first and last row block of every expert (for any block size the kernels use) and its middle
+    hold a checked row; with the number of 128-row blocks covered out of all of them."""
+    counts, offsets, slot_token, _ = oracle.permute(idx.cpu(), E)
+    slots = set()
+    for e in range(E):
+        c, o = int(counts[e]), int(offsets[e])
+        if c:
+            slots.update({o, o + c // 2, o + c - 1})
+    tokens = sorted({int(slot_token[r]) for r in slots})
+    # the 128-row blocks of each expert that the chosen tokens' rows reach
+    tok = torch.zeros(idx.shape[0], dtype=torch.bool)
+    tok[tokens] = True
+    covered, total = 0, 0
+    for e in range(E):
+        c, o = int(counts[e]), int(offsets[e])
+        for b in range((c + 127) // 128):
+            total += 1
+            rows = slot_token[o + 128 * b:o + min(c, 128 * (b + 1))].long()
+            covered += int(tok[rows].any())
+    return tokens, covered, total
 
 
 @pytest.mark.parametrize("name", ["decode", "prefill", "skewed", "block"])
@@ -466,5 +534,11 @@ def test_forward_full_size_sampled(moe, name):
     counts = torch.bincount(idx.cpu().flatten().long(), minlength=w.E)
     assert counts.sum().item() == w.T * w.top_k
     assert torch.isfinite(out).all()
-    tokens = _sample_tokens(w.T, 12, w.seed)
+    # the layer output for tokens that reach the first, middle and last rows of every active expert (every
+    # token of the decode workload), against the oracle
+    tokens, covered, total = _tile_covering_tokens(idx, w.E)
+    if w.T <= 256:
+        tokens = list(range(w.T))
+    print(f"{name}: {len(tokens)} tokens checked; they reach {covered} of {total} 128-row expert blocks, and the "
+          f"first and last block of all {int((counts > 0).sum())} active experts")
     _check_layer(moe, w, I, tokens, result=res)
