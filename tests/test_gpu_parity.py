@@ -500,15 +500,16 @@ def test_forward_launch_count_is_reported_and_stable(moe):
 
 # --------------------------------------------------------------------------- full-size workloads (sampled)
 def _tile_covering_tokens(idx, E):
-    """Tokens whose rows include the first, a middle and the last row of every active expert's segment, so
-    that the first and last row block of every expert (for any block size the kernels use) and its middle
-    hold a checked row; with the number of 128-row blocks covered out of all of them."""
+    """Tokens whose rows include the first row of every 128-row block of every active expert's segment and
+    its last row, so that every row block the kernels use (16 to 256 rows, all aligned to the segment start)
+    holds a checked row; with the number of 128-row blocks covered out of all of them."""
     counts, offsets, slot_token, _ = oracle.permute(idx.cpu(), E)
     slots = set()
     for e in range(E):
         c, o = int(counts[e]), int(offsets[e])
         if c:
-            slots.update({o, o + c // 2, o + c - 1})
+            slots.update(range(o, o + c, 128))
+            slots.add(o + c - 1)
     tokens = sorted({int(slot_token[r]) for r in slots})
     # the 128-row blocks of each expert that the chosen tokens' rows reach
     tok = torch.zeros(idx.shape[0], dtype=torch.bool)
@@ -534,11 +535,12 @@ def test_forward_full_size_sampled(moe, name):
     counts = torch.bincount(idx.cpu().flatten().long(), minlength=w.E)
     assert counts.sum().item() == w.T * w.top_k
     assert torch.isfinite(out).all()
-    # the layer output for tokens that reach the first, middle and last rows of every active expert (every
-    # token of the decode workload), against the oracle
+    # the layer output for tokens that reach every 128-row block and the last row of every active expert
+    # (every token of the decode workload), against the oracle
     tokens, covered, total = _tile_covering_tokens(idx, w.E)
     if w.T <= 256:
         tokens = list(range(w.T))
-    print(f"{name}: {len(tokens)} tokens checked; they reach {covered} of {total} 128-row expert blocks, and the "
-          f"first and last block of all {int((counts > 0).sum())} active experts")
+    print(f"{name}: {len(tokens)} tokens checked; they reach {covered} of {total} 128-row expert blocks of the "
+          f"{int((counts > 0).sum())} active experts")
+    assert covered == total
     _check_layer(moe, w, I, tokens, result=res)
