@@ -60,7 +60,7 @@ namespace tc {
 
 constexpr int BK = 64;  // K elements per stage = one 128-byte swizzle row of bf16
 // warps 0..5 as below; the weights-as-M form adds warps 6..9 that gather activation rows (Args::gather)
-template <bool SWAP>
+template <bool SWAP, bool SWIGLU, int R>
 constexpr int threads_of() { return SWAP ? 320 : 192; }
 constexpr int kSmemLimit = 232448;              // 227 KB opt-in per CTA
 
@@ -94,10 +94,14 @@ struct Cfg {
     static constexpr int TMEM_COLS = (2 * ACC <= 32) ? 32 : (2 * ACC <= 64) ? 64 : (2 * ACC <= 128) ? 128 : (2 * ACC <= 256) ? 256 : 512;
     static_assert(2 * ACC <= 512, "two accumulator buffers must fit in 512 TMEM columns");
     static constexpr int AUX_BYTES = 4096;  // barriers, tile tables
-    static constexpr int STAGES_MAX = (kSmemLimit - 1024 - AUX_BYTES) / STAGE_BYTES;
+    // rows-as-M with 128-row blocks: a 4 KB staging buffer per epilogue warp (32 rows x 64 bf16 columns,
+    // 128-byte swizzle) from which TMA stores the warp's output rows when all 32 are valid
+    static constexpr bool TMA_OUT = !SWAP && R == 128;
+    static constexpr int EPI_BYTES = TMA_OUT ? 4 * 4096 : 0;
+    static constexpr int STAGES_MAX = (kSmemLimit - 1024 - AUX_BYTES - EPI_BYTES) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_MAX > 12 ? 12 : STAGES_MAX;
     static_assert(STAGES >= 2, "pipeline depth");
-    static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + AUX_BYTES;
+    static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + AUX_BYTES + EPI_BYTES;
     static constexpr int LDW = R < 32 ? R : 32;  // TMEM columns per tcgen05.ld in the weights-as-M epilogue
 };
 
@@ -136,6 +140,7 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
+
 struct Aux {  // lives after the stage ring in shared memory
     uint64_t full[12];
     uint64_t empty[12];
@@ -164,9 +169,10 @@ __device__ __forceinline__ void decode_tile(const Aux& a, int E, int R, int tile
 }
 
 template <bool SWAP, bool SWIGLU, int R, int COLS>
-__global__ void __launch_bounds__(threads_of<SWAP>(), 1)
+__global__ void __launch_bounds__(threads_of<SWAP, SWIGLU, R>(), 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_w1,
-                        const __grid_constant__ CUtensorMap tm_w2, const Args p) {
+                        const __grid_constant__ CUtensorMap tm_w2, const __grid_constant__ CUtensorMap tm_out,
+                        const Args p) {
     using C = Cfg<SWAP, SWIGLU, R, COLS>;
     constexpr int STAGES = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
@@ -193,6 +199,7 @@ __global__ void __launch_bounds__(threads_of<SWAP>(), 1)
         tma_prefetch(&tm_act);
         tma_prefetch(&tm_w1);
         if (SWIGLU) tma_prefetch(&tm_w2);
+        if (C::TMA_OUT) tma_prefetch(&tm_out);
     }
     if (warp == 1) tmem_alloc(smem_u32(&aux.tmem_slot), C::TMEM_COLS);
 
@@ -453,47 +460,74 @@ __global__ void __launch_bounds__(threads_of<SWAP>(), 1)
                 const int m = 32 * q + lane;  // activation row inside the tile
                 uint16_t* orow = p.out + (row0 + m) * p.ldo + (int64_t)cb * COLS;
                 const bool valid = m < rows;
+                // a warp whose 32 rows are all valid writes them by TMA from its staging buffer (full 128-byte
+                // rows, no partial-line traffic); a warp with fewer stores its valid rows directly
+                const bool tma_rows = C::TMA_OUT && !p.raw && rows - 32 * q >= 32;
+                const uint32_t stg = smem_u32(smem) + STAGES * C::STAGE_BYTES + C::AUX_BYTES + 4096 * q;
                 // warp-uniform: a lane quarter past the tile's rows holds nothing to store
 #pragma unroll 1
-                for (int c = 0; c < (32 * q < rows ? COLS : 0); c += 32) {
-                    uint32_t g[32];
-                    tmem_ld32(tb + c, g);
-                    uint32_t pk[16];
-                    if constexpr (SWIGLU) {
-                        uint32_t u[32];
-                        tmem_ld32(tb + COLS + c, u);
-                        tmem_wait_ld(g);
-                        tmem_wait_ld(u);
-                        if (p.raw) {  // GEMM-core test form: g and u stored apart
-                            uint32_t pu[16];
+                for (int c = 0; c < (32 * q < rows ? COLS : 0); c += 64) {
+                    uint32_t pk[32];  // 64 bf16 of this lane's row: columns c .. c + 63
 #pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                pk[i] = pack_bf16x2(__uint_as_float(g[2 * i]), __uint_as_float(g[2 * i + 1]));
-                                pu[i] = pack_bf16x2(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1]));
-                            }
-                            if (valid) {
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t g[32];
+                        tmem_ld32(tb + c + 32 * hh, g);
+                        if constexpr (SWIGLU) {
+                            uint32_t u[32];
+                            tmem_ld32(tb + COLS + c + 32 * hh, u);
+                            tmem_wait_ld(g);
+                            tmem_wait_ld(u);
+                            if (p.raw) {  // GEMM-core test form: g and u stored apart
+                                if (valid) {
 #pragma unroll
-                                for (int v = 0; v < 4; ++v) {
-                                    st16(orow + c + 8 * v, make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]));
-                                    st16(orow + p.n_out + c + 8 * v,
-                                         make_uint4(pu[4 * v], pu[4 * v + 1], pu[4 * v + 2], pu[4 * v + 3]));
+                                    for (int v = 0; v < 4; ++v) {
+                                        uint32_t a4[4], b4[4];
+#pragma unroll
+                                        for (int i = 0; i < 4; ++i) {
+                                            a4[i] = pack_bf16x2(__uint_as_float(g[8 * v + 2 * i]),
+                                                                __uint_as_float(g[8 * v + 2 * i + 1]));
+                                            b4[i] = pack_bf16x2(__uint_as_float(u[8 * v + 2 * i]),
+                                                                __uint_as_float(u[8 * v + 2 * i + 1]));
+                                        }
+                                        st16(orow + c + 32 * hh + 8 * v, make_uint4(a4[0], a4[1], a4[2], a4[3]));
+                                        st16(orow + p.n_out + c + 32 * hh + 8 * v,
+                                             make_uint4(b4[0], b4[1], b4[2], b4[3]));
+                                    }
                                 }
+                                continue;
                             }
-                            continue;
-                        }
 #pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            pk[i] = pack_bf16x2(silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
+                            for (int i = 0; i < 16; ++i)
+                                pk[16 * hh + i] =
+                                    pack_bf16x2(silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
                                                 silu_mul(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1])));
-                    } else {
-                        tmem_wait_ld(g);
+                        } else {
+                            tmem_wait_ld(g);
 #pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            pk[i] = pack_bf16x2(__uint_as_float(g[2 * i]), __uint_as_float(g[2 * i + 1]));
+                            for (int i = 0; i < 16; ++i)
+                                pk[16 * hh + i] = pack_bf16x2(__uint_as_float(g[2 * i]), __uint_as_float(g[2 * i + 1]));
+                        }
                     }
-                    if (valid) {
+                    if (SWIGLU && p.raw) continue;
+                    if (tma_rows) {
+                        // the staging buffer is free once the previous store from it has read it
+                        if (lane == 0) bulk_wait_read();
+                        __syncwarp();
+                        // row `lane`, 16-byte chunk v at lane * 128 + ((v ^ (lane % 8)) * 16): the 128-byte swizzle
+                        // of the output tensor map; eight consecutive lanes cover all 32 banks
 #pragma unroll
-                        for (int v = 0; v < 4; ++v)
+                        for (int v = 0; v < 8; ++v)
+                            st_shared16(stg + lane * 128 + ((v ^ (lane & 7)) << 4),
+                                        make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]));
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&tm_out, stg, cb * COLS + c, (int)(row0 + 32 * q));
+                            bulk_commit();
+                        }
+                    } else if (valid) {
+#pragma unroll
+                        for (int v = 0; v < 8; ++v)
                             st16(orow + c + 8 * v, make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]));
                     }
                 }
@@ -539,7 +573,8 @@ __global__ void __launch_bounds__(threads_of<SWAP>(), 1)
         }
     }
 
-    // ---- teardown
+    // ---- teardown: the epilogue's TMA stores are complete before the kernel ends
+    if (C::TMA_OUT && warp >= 2 && warp < 6 && lane == 0) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -574,7 +609,7 @@ static cudaError_t run(const Ctx& c, const void* act, int S, const void* w1, con
         if (err != cudaSuccess) return err;
         attr_done[c.device] = true;
     }
-    CUtensorMap tm_act, tm_w1, tm_w2;
+    CUtensorMap tm_act, tm_w1, tm_w2, tm_out;
     // act holds S permuted rows, or (with a.gather) act_rows rows read through the slot -> row map
     const uint64_t arows = act_rows >= 0 ? (uint64_t)act_rows : (uint64_t)S;
     if (arows == 0) return cudaErrorInvalidValue;
@@ -582,11 +617,14 @@ static cudaError_t run(const Ctx& c, const void* act, int S, const void* w1, con
     if (!encode_2d(&tm_w1, w1, (uint64_t)a.K, (uint64_t)a.E * a.n_out, (uint32_t)C::WBOX)) return cudaErrorInvalidValue;
     if (!encode_2d(&tm_w2, SWIGLU ? w2 : w1, (uint64_t)a.K, (uint64_t)a.E * a.n_out, (uint32_t)C::WBOX))
         return cudaErrorInvalidValue;
+    // the output [S][ldo] in boxes of 64 columns x 32 rows (one epilogue warp's rows), 128-byte swizzle
+    if (!encode_2d(&tm_out, a.out, (uint64_t)a.ldo, (uint64_t)S, 32)) return cudaErrorInvalidValue;
     // upper bound on the tile count: sum_e ceil(cnt_e / R) <= S / R + E
     const int64_t max_tiles = ((int64_t)S / R + a.E) * (a.n_out / COLS);
     const int grid = (int)(max_tiles < c.num_sms ? max_tiles : c.num_sms);
     if (grid <= 0) return cudaSuccess;
-    return launch(kern, dim3(grid), dim3(threads_of<SWAP>()), (size_t)C::SMEM, c, tm_act, tm_w1, tm_w2, a);
+    return launch(kern, dim3(grid), dim3(threads_of<SWAP, SWIGLU, R>()), (size_t)C::SMEM, c, tm_act, tm_w1, tm_w2,
+                  tm_out, a);
 }
 
 // Token rows staged per rows-as-M tile: the smallest of 16/32/64/128 that
@@ -614,8 +652,9 @@ static int pick_swap_rows(int S, int E) {
 
 // Only the weights-as-M gate/up form (few rows per expert) gathers its rows in place: there a tile
 // stages at most 64 rows per K slice, which four gather warps copy well within a stage's time.  For
-// 128-row tiles the gather warps could not keep the ring full (measured: prefill 11% slower than
-// copying the rows once with the permutation), so those read the permuted copy by TMA.
+// 128-row tiles gathering measured slower than copying the rows once with the permutation and
+// reading the copy by TMA: prefill 11% slower with one warp per stage, and still ~5% slower with all
+// four warps filling every stage two cp.async groups ahead, so those read the permuted copy.
 bool gate_up_needs_permuted_rows(int S, int E) { return use_pair_gemm(S, E, 256) || tc::pick_swap_rows(S, E) == 0; }
 
 cudaError_t launch_gate_up_bf16(const Ctx& c, const void* xp, const void* Wg, const void* Wu, const int32_t* counts,

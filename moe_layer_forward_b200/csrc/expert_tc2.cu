@@ -58,7 +58,12 @@ struct Aux2 {
     int cnt[kMaxExperts];
     int off[kMaxExperts];
 };
-constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + (int)sizeof(Aux2);
+constexpr int AUX_BYTES = 4096;
+static_assert((int)sizeof(Aux2) <= AUX_BYTES, "aux block");
+// a 4 KB staging buffer per epilogue warp (32 rows x 64 bf16 columns, 128-byte swizzle) from which TMA stores
+// the warp's output rows when all 32 are valid
+constexpr int EPI_BYTES = 4 * 4096;
+constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + AUX_BYTES + EPI_BYTES;
 static_assert(SMEM <= kSmemLimit, "shared memory budget");
 
 struct Args2 {
@@ -146,7 +151,8 @@ __device__ __forceinline__ void decode_tile2(const Aux2& a, int E, int tile, int
 template <bool SWIGLU>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_w1,
-                            const __grid_constant__ CUtensorMap tm_w2, const Args2 p) {
+                            const __grid_constant__ CUtensorMap tm_w2, const __grid_constant__ CUtensorMap tm_out,
+                            const Args2 p) {
     constexpr int WCOLS = SWIGLU ? 128 : 256;  // output columns of one weight block
     constexpr uint32_t TMEM_COLS = 512;          // two accumulators of up to 256 columns
     extern __shared__ uint8_t smem_raw[];
@@ -174,6 +180,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tma_prefetch(&tm_act);
         tma_prefetch(&tm_w1);
         if (SWIGLU) tma_prefetch(&tm_w2);
+        tma_prefetch(&tm_out);
     }
     cluster_sync();  // the peer's barriers exist before any remote arrive or copy completion
     if (warp == 1) tmem_alloc_pair(smem_u32(&aux.tmem_slot), TMEM_COLS);
@@ -337,49 +344,76 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             uint16_t* orow = p.out + ((int64_t)aux.off[e] + (int64_t)rb * RB + 128 * (int)rank + m) * p.ldo +
                              (int64_t)cb * WCOLS;
             const uint32_t tb_addr = tmem_base + (uint32_t)(buf * 256) + ((uint32_t)(32 * q) << 16);
+            // a warp whose 32 rows are all valid writes them by TMA from its staging buffer (full 128-byte rows);
+            // a warp with fewer stores its valid rows directly
+            const bool tma_rows = !p.raw && rows - 32 * q >= 32;
+            const uint32_t stg = smem_u32(smem) + STAGES * STAGE_BYTES + AUX_BYTES + 4096 * q;
+            const int grow = aux.off[e] + rb * RB + 128 * (int)rank + 32 * q;  // first output row of this warp
             if (rows > 32 * q) {  // skip quarters without valid rows (warp-uniform)
 #pragma unroll 1
-                for (int c = 0; c < WCOLS; c += 32) {
-                    uint32_t g[32];
-                    tmem_ld32(tb_addr + c, g);
-                    uint32_t pk[16];
-                    if constexpr (SWIGLU) {
-                        uint32_t u[32];
-                        tmem_ld32(tb_addr + 128 + c, u);
-                        tmem_wait_ld(g);
-                        tmem_wait_ld(u);
-                        if (p.raw) {  // GEMM-core test form: g and u stored apart
-                            uint32_t pu[16];
+                for (int c = 0; c < WCOLS; c += 64) {
+                    uint32_t pk[32];  // 64 bf16 of this lane's row: columns c .. c + 63
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t g[32];
+                        tmem_ld32(tb_addr + c + 32 * hh, g);
+                        if constexpr (SWIGLU) {
+                            uint32_t u[32];
+                            tmem_ld32(tb_addr + 128 + c + 32 * hh, u);
+                            tmem_wait_ld(g);
+                            tmem_wait_ld(u);
+                            if (p.raw) {  // GEMM-core test form: g and u stored apart
+                                if (valid) {
+#pragma unroll
+                                    for (int v = 0; v < 4; ++v) {
+                                        uint32_t a4[4], b4[4];
+#pragma unroll
+                                        for (int i = 0; i < 4; ++i) {
+                                            a4[i] = pack_bf16x2(__uint_as_float(g[8 * v + 2 * i]),
+                                                                __uint_as_float(g[8 * v + 2 * i + 1]));
+                                            b4[i] = pack_bf16x2(__uint_as_float(u[8 * v + 2 * i]),
+                                                                __uint_as_float(u[8 * v + 2 * i + 1]));
+                                        }
+                                        st16(orow + c + 32 * hh + 8 * v, make_uint4(a4[0], a4[1], a4[2], a4[3]));
+                                        st16(orow + p.n_out + c + 32 * hh + 8 * v,
+                                             make_uint4(b4[0], b4[1], b4[2], b4[3]));
+                                    }
+                                }
+                                continue;
+                            }
 #pragma unroll
                             for (int i = 0; i < 16; ++i) {
-                                pk[i] = pack_bf16x2(__uint_as_float(g[2 * i]), __uint_as_float(g[2 * i + 1]));
-                                pu[i] = pack_bf16x2(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1]));
-                            }
-                            if (valid) {
-#pragma unroll
-                                for (int v = 0; v < 4; ++v) {
-                                    st16(orow + c + 8 * v, make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]));
-                                    st16(orow + p.n_out + c + 8 * v,
-                                         make_uint4(pu[4 * v], pu[4 * v + 1], pu[4 * v + 2], pu[4 * v + 3]));
-                                }
-                            }
-                            continue;
-                        }
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
-                            pk[i] = pack_bf16x2(__fdividef(g0, 1.0f + __expf(-g0)) * __uint_as_float(u[2 * i]),
+                                const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+                                pk[16 * hh + i] =
+                                    pack_bf16x2(__fdividef(g0, 1.0f + __expf(-g0)) * __uint_as_float(u[2 * i]),
                                                 __fdividef(g1, 1.0f + __expf(-g1)) * __uint_as_float(u[2 * i + 1]));
+                            }
+                        } else {
+                            tmem_wait_ld(g);
+#pragma unroll
+                            for (int i = 0; i < 16; ++i)
+                                pk[16 * hh + i] = pack_bf16x2(__uint_as_float(g[2 * i]), __uint_as_float(g[2 * i + 1]));
                         }
-                    } else {
-                        tmem_wait_ld(g);
-#pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            pk[i] = pack_bf16x2(__uint_as_float(g[2 * i]), __uint_as_float(g[2 * i + 1]));
                     }
-                    if (valid) {
+                    if (SWIGLU && p.raw) continue;
+                    if (tma_rows) {
+                        if (lane == 0) bulk_wait_read();  // the previous store from this buffer has read it
+                        __syncwarp();
+                        // row `lane`, 16-byte chunk v at lane * 128 + ((v ^ (lane % 8)) * 16): the output tensor
+                        // map's 128-byte swizzle; eight consecutive lanes cover all 32 banks
 #pragma unroll
-                        for (int v = 0; v < 4; ++v)
+                        for (int v = 0; v < 8; ++v)
+                            st_shared16(stg + lane * 128 + ((v ^ (lane & 7)) << 4),
+                                        make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]));
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&tm_out, stg, cb * WCOLS + c, grow);
+                            bulk_commit();
+                        }
+                    } else if (valid) {
+#pragma unroll
+                        for (int v = 0; v < 8; ++v)
                             st16(orow + c + 8 * v, make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]));
                     }
                 }
@@ -391,7 +425,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (!ok) raise_abort();
     }
 
-    // ---- teardown: the leader's MMAs read this CTA's shared memory and write its tensor memory
+    // ---- teardown: the epilogue's TMA stores are complete; the leader's MMAs read this CTA's shared memory
+    // and write its tensor memory
+    if (warp >= 2 && lane == 0) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
     cluster_sync();
@@ -423,8 +459,10 @@ static cudaError_t run2(const Ctx& c, const void* act, int S, const void* w1, co
         if (err != cudaSuccess) return err;
         attr_done[c.device] = true;
     }
-    CUtensorMap tm_act, tm_w1, tm_w2;
+    CUtensorMap tm_act, tm_w1, tm_w2, tm_out;
     if (!encode(&tm_act, act, (uint64_t)a.K, (uint64_t)S, 128)) return cudaErrorInvalidValue;
+    // the output [S][ldo] in boxes of 64 columns x 32 rows (one epilogue warp's rows)
+    if (!encode(&tm_out, a.out, (uint64_t)a.ldo, (uint64_t)S, 32)) return cudaErrorInvalidValue;
     if (!encode(&tm_w1, w1, (uint64_t)a.K, (uint64_t)a.E * a.n_out, 128)) return cudaErrorInvalidValue;
     if (!encode(&tm_w2, SWIGLU ? w2 : w1, (uint64_t)a.K, (uint64_t)a.E * a.n_out, 128)) return cudaErrorInvalidValue;
     static int max_clusters[64] = {};
@@ -445,7 +483,7 @@ static cudaError_t run2(const Ctx& c, const void* act, int S, const void* w1, co
     int clusters = max_clusters[c.device];
     if (max_tiles < clusters) clusters = (int)max_tiles;
     if (clusters <= 0) return cudaSuccess;
-    return launch(kern, dim3(2 * clusters), dim3(kThreads), (size_t)SMEM, c, tm_act, tm_w1, tm_w2, a);
+    return launch(kern, dim3(2 * clusters), dim3(kThreads), (size_t)SMEM, c, tm_act, tm_w1, tm_w2, tm_out, a);
 }
 
 }  // namespace tc2
