@@ -18,9 +18,9 @@
 //                        then sees the unrounded fp32 normalised row).
 //   router_topk_kernel   one warp per token: sums the K-split partials in split
 //                        order, scores sigmoid(z)+b in fp32 (sigmoid in double,
-//                        rounded once), then k rounds of a warp-shuffle argmax
-//                        over (score, index) packed in 64 bits (ties to the lower
-//                        index) plus one more for the margin.
+//                        rounded once), then k rounds of a warp-wide argmax (two
+//                        warp reductions: the largest score key, then the lowest
+//                        expert index holding it) plus one more for the margin.
 //   router_topk_token_kernel  the same for few tokens: a CTA per token, a thread
 //                        per expert for the split sum, then one warp selects.
 #include <math.h>
@@ -60,6 +60,75 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const void* __restrict__ x
 #pragma unroll
         for (int i = 0; i < 8; ++i) o[i] = (a[i] * r) * g[i];
         store8<VDT>(v, row + j, o);
+    }
+}
+
+// The same with the whole row held in registers (d <= 256 NC): every load of the row is issued before
+// the first is used, so a warp has NC 16-byte loads per lane in flight and x is read once.  Same
+// arithmetic and summation order as rmsnorm_kernel, so the same results bit for bit.
+template <int XDT, int VDT, int NC>
+__global__ void __launch_bounds__(256) rmsnorm_reg_kernel(const void* __restrict__ x, const float* __restrict__ gamma,
+                                                          int T, int d, float eps, void* __restrict__ v,
+                                                          float* __restrict__ rstd_out) {
+    pdl_wait();
+    pdl_trigger();
+    constexpr int V = XDT == DT_BF16 ? 1 : 2;  // 16-byte vectors per 8 elements
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t = (int64_t)blockIdx.x * 8 + warp;
+    if (t >= T) return;
+    const int64_t row = t * d;
+    uint4 raw[NC][V];
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+        const int j = lane * 8 + c * 256;
+        if (j < d) {
+#pragma unroll
+            for (int q = 0; q < V; ++q)
+                raw[c][q] = XDT == DT_BF16 ? ld16(static_cast<const uint16_t*>(x) + row + j)
+                                           : ld16(static_cast<const float*>(x) + row + j + 4 * q);
+        }
+    }
+    auto unpack = [&](int c, float (&a)[8]) {
+        if constexpr (XDT == DT_BF16) {
+            const uint32_t wv[4] = {raw[c][0].x, raw[c][0].y, raw[c][0].z, raw[c][0].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                a[2 * i] = bf16_bits_to_f32(wv[i] & 0xFFFFu);
+                a[2 * i + 1] = bf16_bits_to_f32(wv[i] >> 16);
+            }
+        } else {
+            a[0] = __uint_as_float(raw[c][0].x); a[1] = __uint_as_float(raw[c][0].y);
+            a[2] = __uint_as_float(raw[c][0].z); a[3] = __uint_as_float(raw[c][0].w);
+            a[4] = __uint_as_float(raw[c][V - 1].x); a[5] = __uint_as_float(raw[c][V - 1].y);
+            a[6] = __uint_as_float(raw[c][V - 1].z); a[7] = __uint_as_float(raw[c][V - 1].w);
+        }
+    };
+    float ss = 0.f;
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+        if (lane * 8 + c * 256 < d) {
+            float a[8];
+            unpack(c, a);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) ss = fmaf(a[i], a[i], ss);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float r = 1.0f / sqrtf(ss / (float)d + eps);
+    if (lane == 0 && rstd_out) rstd_out[t] = r;
+    if (v == nullptr) return;
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+        const int j = lane * 8 + c * 256;
+        if (j < d) {
+            float a[8], g[8], o[8];
+            unpack(c, a);
+            load8<DT_F32>(gamma, j, g);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) o[i] = (a[i] * r) * g[i];
+            store8<VDT>(v, row + j, o);
+        }
     }
 }
 
@@ -105,7 +174,11 @@ static cudaError_t launch_rms(const Ctx& c, const void* x, const float* gamma, i
                               float* rstd) {
     if (T <= 2 * 8 * c.num_sms)  // fewer rows than two waves of warp-per-row CTAs
         return launch(rmsnorm_row_kernel<XDT, VDT>, dim3(T), dim3(256), 0, c, x, gamma, T, d, eps, v, rstd);
-    return launch(rmsnorm_kernel<XDT, VDT>, dim3((T + 7) / 8), dim3(256), 0, c, x, gamma, T, d, eps, v, rstd);
+    const dim3 g((T + 7) / 8);
+    if (d <= 1024) return launch(rmsnorm_reg_kernel<XDT, VDT, 4>, g, dim3(256), 0, c, x, gamma, T, d, eps, v, rstd);
+    if (d <= 2048) return launch(rmsnorm_reg_kernel<XDT, VDT, 8>, g, dim3(256), 0, c, x, gamma, T, d, eps, v, rstd);
+    if (d <= 4096) return launch(rmsnorm_reg_kernel<XDT, VDT, 16>, g, dim3(256), 0, c, x, gamma, T, d, eps, v, rstd);
+    return launch(rmsnorm_kernel<XDT, VDT>, g, dim3(256), 0, c, x, gamma, T, d, eps, v, rstd);
 }
 
 cudaError_t launch_rmsnorm(const Ctx& c, const void* x, int x_dt, const float* gamma, int T, int d, float eps, void* v,
@@ -119,8 +192,9 @@ cudaError_t launch_rmsnorm(const Ctx& c, const void* x, int x_dt, const float* g
 
 // ----------------------------------------------------------------------------- top-k
 // Scores, top-k selection and weights of token t from its logits z[j] = z(lane + 32 j), by one
-// warp: sigmoid in double rounded once to fp32, + b in fp32, k rounds of a warp-shuffle argmax
-// (ties to the lower index) and one more for the margin to the first expert left out.
+// warp: sigmoid in double rounded once to fp32, + b in fp32, k rounds of a warp-wide argmax (a max
+// reduction of the order-preserving score keys, then a min reduction of the expert indices holding
+// the maximum: ties go to the lower index) and one more for the margin to the first expert left out.
 // Order-preserving 32-bit image of a non-NaN float (a larger float gives a larger unsigned; -0 is +0).
 __device__ __forceinline__ uint32_t ordered_bits(float f) {
     const uint32_t u = __float_as_uint(f + 0.0f);
@@ -129,39 +203,34 @@ __device__ __forceinline__ uint32_t ordered_bits(float f) {
 __device__ __forceinline__ float from_ordered(uint32_t o) {
     return __uint_as_float((o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o);
 }
-__device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t v, int o) {
-    const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, o);
-    const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v >> 32), o);
-    return ((uint64_t)hi << 32) | lo;
-}
-
 __device__ __forceinline__ void select_topk_warp(const float (&z)[8], int lane, int t, const float* __restrict__ b,
                                                  int E, int k, int32_t* __restrict__ idx, float* __restrict__ w,
                                                  float* __restrict__ logits, float* __restrict__ margin) {
-    // candidate of entry e = lane + 32 j: (ordered score << 32) | ~e, so that the largest value is the
-    // highest score and, among equal scores, the lowest expert index; 0 = no candidate
-    uint64_t cand[8];
+    // key of entry e = lane + 32 j: the order-preserving image of its score (NaN as -inf), 0 = no candidate
+    uint32_t key[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         const int e = lane + 32 * j;
-        cand[j] = 0;
+        key[j] = 0;
         if (e < E) {
             const float acc = z[j];
             if (logits) logits[(int64_t)t * E + e] = acc;
             const float sg = (float)(1.0 / (1.0 + exp(-(double)acc)));
             const float sc = sg + b[e];
-            cand[j] = ((uint64_t)ordered_bits(isnan(sc) ? -INFINITY : sc) << 32) | (0xFFFFFFFFu - (uint32_t)e);
+            key[j] = ordered_bits(isnan(sc) ? -INFINITY : sc);
         }
     }
-    // this lane's best remaining candidate and its logit
-    uint64_t best = 0;
+    // this lane's best remaining entry (largest key, the lowest expert index among equal keys) and its logit
+    uint32_t best = 0;
+    int best_e = 0;
     float best_z = 0.f;
     auto refresh = [&]() {
         best = 0;
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-            if (cand[j] > best) {
-                best = cand[j];
+            if (key[j] > best) {
+                best = key[j];
+                best_e = lane + 32 * j;
                 best_z = z[j];
             }
     };
@@ -170,17 +239,13 @@ __device__ __forceinline__ void select_topk_warp(const float (&z)[8], int lane, 
     float sel_z[kMaxTopK];
     float kth = 0.f, next = INFINITY;
     const int rounds = k + (E > k ? 1 : 0);
+    // each round: the warp's largest key (one reduction), then the lowest expert index holding it (a second)
 #pragma unroll
     for (int r = 0; r < kMaxTopK + 1; ++r) {
         if (r >= rounds) break;
-        uint64_t m = best;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const uint64_t v = shfl_xor_u64(m, o);
-            m = v > m ? v : m;
-        }
-        const int be = (int)(0xFFFFFFFFu - (uint32_t)m);
-        const float bk = from_ordered((uint32_t)(m >> 32));
+        const uint32_t m = __reduce_max_sync(0xffffffffu, best);
+        const int be = (int)__reduce_min_sync(0xffffffffu, best == m ? (uint32_t)best_e : 0xFFFFFFFFu);
+        const float bk = from_ordered(m);
         if (r < k) {
             sel_z[r] = __shfl_sync(0xffffffffu, best_z, be & 31);
             sel_e[r] = be;
@@ -188,7 +253,7 @@ __device__ __forceinline__ void select_topk_warp(const float (&z)[8], int lane, 
             if ((be & 31) == lane) {  // the winner's lane drops it and finds its next best
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
-                    if (j == (be >> 5)) cand[j] = 0;
+                    if (j == (be >> 5)) key[j] = 0;
                 refresh();
             }
         } else {

@@ -70,10 +70,16 @@ __global__ void __launch_bounds__(256) perm_scan_kernel(int32_t* __restrict__ hi
     const int e = threadIdx.x;
     int run = 0;
     if (e < E) {
-        for (int c = 0; c < nchunks; ++c) {
-            const int v = hist[(int64_t)c * E + e];
-            hist[(int64_t)c * E + e] = run;
-            run += v;
+        // batches of 16 chunks: the loads of a batch are independent and in flight together
+        for (int c0 = 0; c0 < nchunks; c0 += 16) {
+            int v[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] = c0 + i < nchunks ? hist[(int64_t)(c0 + i) * E + e] : 0;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                if (c0 + i < nchunks) hist[(int64_t)(c0 + i) * E + e] = run;
+                run += v[i];
+            }
         }
         counts[e] = run;
     }
