@@ -315,8 +315,8 @@ class Layer:
 
 
 def near_ties(L) -> dict:
-    """Tokens whose 8th-to-9th selection-score margin is below 1e-5, from the library's own router (fp32
-    normalised rows, as moe_forward routes them); a diagnostic, outside every timed region."""
+    """Tokens whose 8th-to-9th selection-score margin is below 1e-5, from the library's routing of the layer
+    (moe_route: the forward's own router, bit for bit); a diagnostic, outside every timed region."""
     import torch
 
     import moe_layer_forward_b200 as moe
@@ -324,15 +324,12 @@ def near_ties(L) -> dict:
     w, D, dev = L.w, L.D, L.dev
     if w.E <= w.top_k:
         return {"count": 0, "threshold": 1e-5, "tokens": w.T}
-    v32 = torch.empty((w.T, w.d), dtype=torch.float32, device=dev)
-    moe.moe_rmsnorm(D["x"], D["gamma"], w.eps, v32)
     idx = torch.empty((w.T, w.top_k), dtype=torch.int32, device=dev)
     wt = torch.empty((w.T, w.top_k), dtype=torch.float32, device=dev)
     margin = torch.empty(w.T, dtype=torch.float32, device=dev)
-    moe.moe_router_topk(v32, D["W_r"], D["b"], idx, wt, margin=margin)
+    moe.moe_route(D["x"], D["gamma"], D["W_r"], D["b"], idx, wt, w.eps, margin=margin)
     n = int((margin < 1e-5).sum().item())
-    return {"count": n, "threshold": 1e-5, "tokens": w.T,
-            "same_routing_as_forward": bool(torch.equal(idx, L.idx))}
+    return {"count": n, "threshold": 1e-5, "tokens": w.T, "routing_equals_forward": bool(torch.equal(idx, L.idx))}
 
 
 def staged(L, a, barrier, pk) -> tuple:

@@ -124,6 +124,25 @@ moe_status_t moe_router_topk(const void* v, moe_dtype_t v_dt, const float* W_r, 
                              float* margin, void* ws, size_t* ws_bytes, moe_stream_t stream);
 
 /*
+ * Steps 1-2 as the whole layer runs them [P1 §Norm&Residual and §MoE Router
+ * 过程]: the router on the RMSNorm of x without materialising it,
+ *   z = rstd * (x (gamma ⊙ W_r)^T),  rstd = 1 / sqrt((1/d) sum_k x_k^2 + eps),
+ * then selection and weights as in moe_router_topk.  The same kernels as
+ * moe_forward's first steps, so the routing is moe_forward's bit for bit
+ * (a caller that runs the rest of the layer itself, e.g. with experts on
+ * several ranks, routes exactly as the single-GPU layer).  With bf16 x and
+ * d % 128 == 0 gamma ⊙ W_r is rounded once to fp32 and split exactly into
+ * three bf16 terms, so the logits are fp32-accurate sums of exact products;
+ * otherwise the normalised rows are formed in fp32 and multiplied in 3xTF32.
+ * x [T][d] (x_dt), gamma [d], W_r [E][d], b [E]; outputs as moe_router_topk.
+ * Workspace: 1/rms per token, the split-K partial logits and the split
+ * weights.  Requires 1 <= k <= 8, k <= E <= 256, d % 8 == 0.
+ */
+moe_status_t moe_route(const void* x, moe_dtype_t x_dt, const float* gamma, const float* W_r, const float* b,
+                       int32_t T, int32_t d, int32_t E, int32_t k, float eps, int32_t* topk_idx, float* topk_w,
+                       float* logits, float* margin, void* ws, size_t* ws_bytes, moe_stream_t stream);
+
+/*
  * Step 3 — token permutation into expert-contiguous rows
  * [P5 §Token 分发策略, token_permutation; §专家计算实现, contiguous layout]:
  *   counts[e]      = number of (t, i) with topk_idx[t][i] == e

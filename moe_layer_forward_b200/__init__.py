@@ -48,6 +48,7 @@ class MoeWeightsFP8(ctypes.Structure):
 _sig = {
     "moe_rmsnorm": [_vp, _i32, _vp, _i32, _i32, _f32, _vp, _i32, _vp],
     "moe_router_topk": [_vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _szp, _vp],
+    "moe_route": [_vp, _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp, _vp, _vp, _szp, _vp],
     "moe_permute": [_vp, _i32, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _szp, _vp, _vp],
     "moe_permute_static_ws": [_vp, _i32, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
     "moe_expert_gate_up": [_vp, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp],
@@ -154,6 +155,22 @@ def moe_router_topk(v, W_r, b, topk_idx, topk_w, logits=None, margin=None, ws=No
         ws = _ws(lambda w, n: _check("moe_router_topk", call(w, n)), v.device)
     n = ctypes.c_size_t(ws.numel())
     _check("moe_router_topk", call(_p(ws), ctypes.byref(n)))
+
+
+def moe_route(x, gamma, W_r, b, topk_idx, topk_w, eps: float = 1e-5, logits=None, margin=None, ws=None) -> None:
+    """RMSNorm + router top-k of x exactly as moe_forward runs them (the normalised rows are not materialised)."""
+    T, d = x.shape
+    E = W_r.shape[0]
+    k = topk_idx.shape[1]
+
+    def call(wsp, nbytes):
+        return _lib.moe_route(_p(x), _dt(x), _p(gamma), _p(W_r), _p(b), T, d, E, k, eps, _p(topk_idx), _p(topk_w),
+                              _p(logits), _p(margin), wsp, nbytes, _stream(x.device))
+
+    if ws is None:
+        ws = _ws(lambda w, n: _check("moe_route", call(w, n)), x.device)
+    n = ctypes.c_size_t(ws.numel())
+    _check("moe_route", call(_p(ws), ctypes.byref(n)))
 
 
 def moe_permute(v, topk_idx, E: int, counts, offsets, slot_token, token_slot, xp, ws=None, dev_status=None) -> None:

@@ -170,6 +170,37 @@ moe_status_t moe_router_topk(const void* v, moe_dtype_t v_dt, const float* W_r, 
     return cuda_status(launch_router_topk(c, plan, partial, b, T, E, k, topk_idx, topk_w, logits, margin));
 }
 
+moe_status_t moe_route(const void* x, moe_dtype_t x_dt, const float* gamma, const float* W_r, const float* b,
+                       int32_t T, int32_t d, int32_t E, int32_t k, float eps, int32_t* topk_idx, float* topk_w,
+                       float* logits, float* margin, void* ws, size_t* ws_bytes, moe_stream_t stream) {
+    moe_status_t st = check_router_shape(T, d, E, k);
+    if (st != MOE_OK) return st;
+    if (!valid_dt(x_dt)) return MOE_ERR_INVALID_ARG;
+    Ctx c;
+    st = make_ctx(stream, c);
+    if (st != MOE_OK) return st;
+    const RouterPlan plan = plan_router(T, d, E, c.num_sms);
+    Carve cv(nullptr);
+    cv.take((size_t)T * sizeof(float));
+    cv.take(plan.partial_bytes);
+    cv.take(plan.wsplit_bytes);
+    bool query = false;
+    st = check_ws(ws, ws_bytes, cv.off, &query);
+    if (st != MOE_OK || query || T == 0) return st;
+    if (!x || !gamma || !W_r || !b || !topk_idx || !topk_w || !aligned16(x) || !aligned16(gamma) || !aligned16(W_r))
+        return MOE_ERR_INVALID_ARG;
+    Carve w(ws);
+    float* rstd = static_cast<float*>(w.take((size_t)T * sizeof(float)));
+    float* partial = static_cast<float*>(w.take(plan.partial_bytes));
+    float* wsplit = static_cast<float*>(w.take(plan.wsplit_bytes));
+    // the same kernels, in the same order, as steps 1-2 of moe_forward (1/rms only: no normalised copy)
+    st = cuda_status(launch_rmsnorm(c, x, x_dt, gamma, T, d, eps, nullptr, MOE_F32, rstd));
+    if (st != MOE_OK) return st;
+    st = cuda_status(launch_router_logits(c, plan, x, x_dt, rstd, gamma, W_r, T, d, E, partial, wsplit, nullptr));
+    if (st != MOE_OK) return st;
+    return cuda_status(launch_router_topk(c, plan, partial, b, T, E, k, topk_idx, topk_w, logits, margin));
+}
+
 moe_status_t moe_permute(const void* v, moe_dtype_t v_dt, const int32_t* topk_idx, int32_t T, int32_t d, int32_t E,
                          int32_t k, int32_t* counts, int32_t* offsets, int32_t* slot_token, int32_t* token_slot,
                          void* xp, void* ws, size_t* ws_bytes, int32_t* dev_status, moe_stream_t stream) {

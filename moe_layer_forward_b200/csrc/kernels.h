@@ -68,6 +68,11 @@ RouterPlan plan_router(int T, int d, int E, int num_sms);
 cudaError_t launch_router_logits(const Ctx& c, const RouterPlan& p, const void* a, int a_dt, const float* rstd,
                                  const float* gamma, const float* W_r, int T, int d, int E, float* partial,
                                  float* wsplit, int32_t* status);
+// bf16 x with rstd (d % 128 == 0): z = rstd * (x (gamma ⊙ W_r)^T) with gamma ⊙ W_r split exactly into three
+// bf16 terms (router_x3.cu); ws holds the split weights (3 E d bf16, within wsplit_bytes)
+cudaError_t launch_router_logits_x3(const Ctx& c, const RouterPlan& p, const void* x, const float* rstd,
+                                    const float* gamma, const float* W_r, int T, int d, int E, int np,
+                                    float* partial, void* ws, int32_t* status);
 cudaError_t launch_router_topk(const Ctx& c, const RouterPlan& p, const float* partial, const float* b, int T, int E,
                                int k, int32_t* idx, float* w, float* logits, float* margin);
 

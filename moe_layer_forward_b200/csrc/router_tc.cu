@@ -456,6 +456,9 @@ cudaError_t launch_router_logits(const Ctx& c, const RouterPlan& p, const void* 
                                  const float* gamma, const float* W_r, int T, int d, int E, float* partial,
                                  float* wsplit, int32_t* status) {
     if (T == 0) return cudaSuccess;
+    // bf16 rows with the normalisation folded in: three exact bf16 MMAs per K step on x itself
+    if (rstd != nullptr && a_dt == DT_BF16 && d % 128 == 0)
+        return launch_router_logits_x3(c, p, a, rstd, gamma, W_r, T, d, E, block_experts(E), partial, wsplit, status);
     float* whi = wsplit;
     float* wlo = wsplit + (size_t)E * d;
     const int64_t n = (int64_t)E * d;

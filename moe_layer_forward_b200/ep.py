@@ -53,6 +53,15 @@ class CudaOps:
         self.m.moe_rmsnorm(x, gamma, eps, v)
         return v
 
+    def route(self, x, gamma, eps, W_r, b, k):
+        """the routing of moe_forward (RMSNorm folded into the router), bit for bit"""
+        T = x.shape[0]
+        idx = torch.empty((T, k), dtype=torch.int32, device=x.device)
+        w = torch.empty((T, k), dtype=torch.float32, device=x.device)
+        if T > 0:
+            self.m.moe_route(x, gamma, W_r, b, idx, w, eps)
+        return idx, w
+
     def router(self, v32, W_r, b, k):
         T = v32.shape[0]
         idx = torch.empty((T, k), dtype=torch.int32, device=v32.device)
@@ -110,9 +119,8 @@ def ep_forward(x, gamma, W_r, b, W_gate_local, W_up_local, W_down_local, E: int,
     d = x.shape[1]
 
     # 1-3: local routing and dispatch order
-    v32 = ops.rmsnorm(x, gamma, eps, torch.float32)
     vx = ops.rmsnorm(x, gamma, eps, W_gate_local.dtype)
-    idx, w = ops.router(v32, W_r, b, top_k)
+    idx, w = ops.route(x, gamma, eps, W_r, b, top_k)
     counts, _, token_slot, xp = ops.permute(vx, idx, E)
 
     # 4: counts, then rows

@@ -154,9 +154,8 @@ class _Route:
 
 
 def _route(ops, x, gamma, W_r, b, E, top_k, eps, dtype) -> _Route:
-    v32 = ops.rmsnorm(x, gamma, eps, torch.float32)
     vx = ops.rmsnorm(x, gamma, eps, dtype)
-    idx, w = ops.router(v32, W_r, b, top_k)
+    idx, w = ops.route(x, gamma, eps, W_r, b, top_k)
     counts, offsets, token_slot = ops.permute_maps(vx, idx, E)
     return _Route(idx, w, vx, counts, offsets, token_slot)
 

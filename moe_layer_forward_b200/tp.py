@@ -43,9 +43,8 @@ def tp_forward(x, gamma, W_r, b, W_gate_slice, W_up_slice, W_down_slice, top_k: 
     out_dtype = out_dtype or x.dtype
     if W_down_slice.shape[2] != W_gate_slice.shape[1]:
         raise ValueError("W_down's slice must match the gate/up feature slice")
-    v32 = ops.rmsnorm(x, gamma, eps, torch.float32)
     vx = ops.rmsnorm(x, gamma, eps, W_gate_slice.dtype)
-    idx, w = ops.router(v32, W_r, b, top_k)
+    idx, w = ops.route(x, gamma, eps, W_r, b, top_k)
     counts, offsets, token_slot, xp = ops.permute(vx, idx, E)
     y_part = ops.grouped_swiglu(xp, W_gate_slice, W_up_slice, W_down_slice, counts, offsets)
     residual = x if rank == 0 else torch.zeros_like(x)
@@ -70,9 +69,8 @@ def tp_partials_emulated(x, gamma, W_r, b, W_gate, W_up, W_down, N: int, top_k: 
     if d_ff % N != 0 or (d_ff // N) % 128 != 0:
         raise ValueError(f"d_ff = {d_ff} does not split over {N} ranks in multiples of 128")
     F = d_ff // N
-    v32 = ops.rmsnorm(x, gamma, eps, torch.float32)
     vx = ops.rmsnorm(x, gamma, eps, W_gate.dtype)
-    idx, w = ops.router(v32, W_r, b, top_k)
+    idx, w = ops.route(x, gamma, eps, W_r, b, top_k)
     counts, offsets, token_slot, xp = ops.permute(vx, idx, E)
     parts = []
     for r in range(N):

@@ -38,6 +38,9 @@ class OracleOps:
         idx, w, _ = self.o.select_topk(z.float(), b, k)
         return idx, w.float()
 
+    def route(self, x, gamma, eps, W_r, b, k):
+        return self.router(self.rmsnorm(x, gamma, eps, torch.float32), W_r, b, k)
+
     def permute(self, v, idx, E):
         counts, offsets, slot_token, token_slot = self.o.permute(idx, E)
         return counts, offsets, token_slot, v[slot_token.long()]

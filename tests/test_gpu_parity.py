@@ -79,6 +79,37 @@ def test_router_topk(moe, T, d, E, k, vdt):
         assert torch.isinf(margin.cpu()).all()
 
 
+@pytest.mark.parametrize("T,d,E,k,xdt", [(300, 512, 32, 8, "bf16"), (129, 4096, 128, 8, "bf16"), (64, 256, 256, 8, "bf16"),
+                                         (70, 264, 16, 2, "bf16"), (90, 512, 64, 8, "f32"), (1, 1024, 128, 8, "bf16")])
+def test_route_is_the_forward_routing_and_matches_the_oracle(moe, T, d, E, k, xdt):
+    # moe_route: RMSNorm folded into the router (bf16 x with d % 128 == 0: three exact bf16 products per
+    # step; otherwise normalised rows in 3xTF32); logits within 1e-4 of the fp64 oracle, routing bit-exact
+    # given them, and identical to what moe_forward routes
+    x = synth.normal((T, d), 250 + E, 1, dtype=DT[xdt])
+    gamma = synth.normal((d,), 250 + E, 4, 1.0, math.sqrt(0.1))
+    W_r = synth.normal((E, d), 250 + E, 2, 0.0, 1 / math.sqrt(d))
+    b = synth.uniform((E,), 250 + E, 3, -0.1, 0.1)
+    idx = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    w = torch.empty((T, k), dtype=torch.float32, device=DEV)
+    logits = torch.empty((T, E), dtype=torch.float32, device=DEV)
+    margin = torch.empty(T, dtype=torch.float32, device=DEV)
+    moe.moe_route(cuda(x), cuda(gamma), cuda(W_r), cuda(b), idx, w, 1e-5, logits=logits, margin=margin)
+    z_ref = oracle.router_logits(oracle.rmsnorm(x, gamma, 1e-5), W_r)
+    assert (logits.cpu().double() - z_ref).abs().max().item() < 1e-4
+    check_routing(oracle, logits, b, idx, w, k)
+    _, _, m_ref = oracle.select_topk(logits.cpu(), b, k)
+    assert torch.equal(margin.cpu(), m_ref)
+    if d % 128 == 0:  # the layer itself (bf16 experts need d % 128 == 0)
+        d_ff = 128
+        Wg = cuda(synth.normal((E, d_ff, d), 251, 5, 0.0, 1 / math.sqrt(d), torch.bfloat16))
+        Wd = cuda(synth.normal((E, d, d_ff), 251, 7, 0.0, 1 / math.sqrt(d_ff), torch.bfloat16))
+        out = torch.empty((T, d), dtype=DT[xdt], device=DEV)
+        i2, w2 = torch.empty_like(idx), torch.empty_like(w)
+        moe.moe_forward(cuda(x), cuda(gamma), cuda(W_r), cuda(b), Wg, Wg, Wd, out, top_k=k, topk_idx=i2, topk_w=w2)
+        torch.cuda.synchronize()
+        assert torch.equal(i2, idx) and torch.equal(w2, w)
+
+
 def test_router_all_equal_scores_pick_lowest_indices(moe):
     T, d, E = 20, 256, 64
     v = torch.zeros((T, d), device=DEV)

@@ -56,11 +56,9 @@ def test_sliced_tensor_parallel_partials_sum_to_the_layer(moe, N, shape):
         block = torch.stack([p[rows] for p in parts]).sum(0)
         b_abs, b_rel = errors(block.to(w.out_dtype), ref[rows])
         assert b_abs <= MAX_ABS and b_rel <= REL_L2, (r, b_abs, b_rel)
-    # the routing is the single-GPU router's, bit-exact given its logits
+    # the routing is the single-GPU layer's (moe_route), bit-exact given its logits
     logits = torch.empty((T, E), dtype=torch.float32, device=DEV)
-    v32 = torch.empty((T, d), dtype=torch.float32, device=DEV)
-    moe.moe_rmsnorm(D["x"], D["gamma"], w.eps, v32)
     i2, w2 = torch.empty_like(idx), torch.empty_like(wt)
-    moe.moe_router_topk(v32, D["W_r"], D["b"], i2, w2, logits=logits)
+    moe.moe_route(D["x"], D["gamma"], D["W_r"], D["b"], i2, w2, w.eps, logits=logits)
     assert torch.equal(i2, idx) and torch.equal(w2, wt)
     check_routing(oracle, logits, I["b"], idx, wt, w.top_k)
