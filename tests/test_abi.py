@@ -212,3 +212,23 @@ def test_forward_rejects_bad_shapes_on_host(lib):
         assert f(ctypes.byref(s), w, NULL, NULL, NULL, NULL, NULL, NULL, ctypes.byref(n), NULL, NULL) == UNSUPPORTED
     s = Shape(8, 4096, 128, 8, 1536, 1e-5, 3, 1, 1)
     assert f(ctypes.byref(s), w, NULL, NULL, NULL, NULL, NULL, NULL, ctypes.byref(n), NULL, NULL) == INVALID
+
+
+def test_route_and_gate_up_raw_reject_bad_arguments_on_host(lib):
+    i32, V = ctypes.c_int32, ctypes.c_void_p
+    r = lib.moe_route
+    r.argtypes = [V, ctypes.c_int, V, V, V, i32, i32, i32, i32, ctypes.c_float, V, V, V, V, V,
+                  ctypes.POINTER(ctypes.c_size_t), V]
+    n = ctypes.c_size_t(0)
+    p = ctypes.c_void_p(16)
+    assert r(p, 1, p, p, p, 8, 4096, 128, 9, 1e-5, p, p, None, None, None, ctypes.byref(n), None) == UNSUPPORTED
+    assert r(p, 1, p, p, p, 8, 4096, 512, 8, 1e-5, p, p, None, None, None, ctypes.byref(n), None) == UNSUPPORTED
+    assert r(p, 1, p, p, p, 8, 4100, 128, 8, 1e-5, p, p, None, None, None, ctypes.byref(n), None) == UNSUPPORTED
+    assert r(p, 3, p, p, p, 8, 4096, 128, 8, 1e-5, p, p, None, None, None, ctypes.byref(n), None) == INVALID
+    assert r(p, 1, p, p, p, -1, 4096, 128, 8, 1e-5, p, p, None, None, None, ctypes.byref(n), None) == INVALID
+    g = lib.moe_expert_gate_up_raw
+    g.argtypes = [V, V, V, V, V, i32, i32, i32, i32, V, V, V]
+    assert g(p, p, p, p, p, 64, 8, 4000, 1536, p, None, None) == UNSUPPORTED  # bf16 needs d % 128
+    assert g(p, p, p, p, p, -1, 8, 4096, 1536, p, None, None) == INVALID
+    assert g(p, None, p, p, p, 64, 8, 4096, 1536, p, None, None) == INVALID
+    assert g(p, p, p, p, p, 0, 8, 4096, 1536, p, None, None) == OK  # no rows: nothing to do
