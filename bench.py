@@ -391,6 +391,10 @@ def staged(L, a, barrier, pk) -> tuple:
                 "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = traffic_for(w.name)
+    if roof["traffic"] is not None:
+        roof["traffic_note"] = ("DRAM bytes of the same kernel template as run by moe_forward, which gathers the "
+                                "token rows from V instead of reading the permuted copy Xp timed here (S*d*2 - "
+                                "T*d*2 fewer algorithmic bytes)")
     roof["kernel"] = "grouped_gemm_kernel (expert gate/up + SwiGLU)"
     roof["algorithmic_bytes_per_launch"] = gate_up_bytes
     roof["algorithmic_flops_per_launch"] = gate_up_flops

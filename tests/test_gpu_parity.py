@@ -79,8 +79,11 @@ def test_router_topk(moe, T, d, E, k, vdt):
         assert torch.isinf(margin.cpu()).all()
 
 
+# bf16 cases cover an expert count that is not a multiple of the 64-expert block (E = 40) and, with T = 640 at
+# d = 4096, K splits of two 128-column chunks each of which the last ten are empty (their partial sums are zero)
 @pytest.mark.parametrize("T,d,E,k,xdt", [(300, 512, 32, 8, "bf16"), (129, 4096, 128, 8, "bf16"), (64, 256, 256, 8, "bf16"),
-                                         (70, 264, 16, 2, "bf16"), (90, 512, 64, 8, "f32"), (1, 1024, 128, 8, "bf16")])
+                                         (70, 264, 16, 2, "bf16"), (90, 512, 64, 8, "f32"), (1, 1024, 128, 8, "bf16"),
+                                         (50, 256, 40, 8, "bf16"), (640, 4096, 128, 8, "bf16")])
 def test_route_is_the_forward_routing_and_matches_the_oracle(moe, T, d, E, k, xdt):
     # moe_route: RMSNorm folded into the router (bf16 x with d % 128 == 0: three exact bf16 products per
     # step; otherwise normalised rows in 3xTF32); logits within 1e-4 of the fp64 oracle, routing bit-exact
