@@ -90,3 +90,19 @@ def test_reference_arm_runs_only_on_rank_zero(monkeypatch):
     monkeypatch.setenv("WORLD_SIZE", "2")
     a = argparse.Namespace(steps=2, warmup=3, gpus=2)
     assert bench.run_reference(a, synth.WORKLOADS["decode"]) == 0  # returns at once, no inputs generated
+
+
+def test_clock_summary_decodes_throttle_reasons():
+    # the bench's clock record from NVML samples (SM MHz, clocks-event reason bits, W): the median clock, the
+    # union of the reasons that reject or annotate a run, and how many samples it rests on
+    sys.path.insert(0, ROOT)
+    import bench
+
+    c = bench.Clocks(0)
+    c.thread = object()  # as if the NVML sampler had run
+    c.max_mhz = 1965.0
+    c.samples = [(1965, 0x0, 700.0), (1500, 0x4, 990.0), (1400, 0x4 | 0x1, 1000.0), (1800, 0x40, 950.0)]
+    s = c.summary()
+    assert s["sm_mhz"] == 1650.0 and s["sm_min_mhz"] == 1400 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+    assert s["samples"] == 4 and s["power_w"] == 970.0
