@@ -54,6 +54,8 @@ def parse():
                          "for ncu captures of the same kernels, never for reported numbers")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-anchor", action="store_true",
+                    help="skip the comparison of the expert GEMMs with a vendor grouped GEMM (bf16 workloads)")
     ap.add_argument("--no-ep", action="store_true", help="skip the one-rank expert-parallel (peer memory) timing")
     ap.add_argument("--no-fp8", action="store_true",
                     help="skip the block-FP8 layer timing (run for bf16 workloads of <= 32 rows per expert)")
@@ -549,6 +551,62 @@ def headline_extras(L, a, barrier, pk, ms_per_step, staged_bufs, active) -> dict
     return res
 
 
+def vendor_anchor(L, a, bufs, local) -> dict | None:
+    """The expert GEMMs of this library against a vendor grouped GEMM (torch.nn.functional.grouped_mm, a CUTLASS
+    kernel) on the same permuted rows, weights and expert segments. Each timing is 3 untimed and 10 timed calls
+    after a 0.5 s idle gap, so both run at the burst clock; medians over 3 interleaved rounds. The vendor call
+    multiplies the gate and up weights as one fused N = 2 d_ff operand and applies no SwiGLU. Outside the
+    timed region; a comparison only, nothing of the layer runs through it."""
+    import torch
+
+    import moe_layer_forward_b200 as moe
+
+    w, D, dev = L.w, L.D, L.dev
+    F = torch.nn.functional
+    if w.w_dtype != torch.bfloat16 or not hasattr(F, "grouped_mm"):
+        return None
+    counts, offsets, xp = bufs
+    S = w.T * w.top_k
+    ends = offsets[1:].contiguous()
+    wgu = torch.cat([D["W_gate"], D["W_up"]], 1)
+    h = torch.empty((S, w.d_ff), dtype=w.w_dtype, device=dev)
+    y = torch.empty((S, w.d), dtype=w.w_dtype, device=dev)
+    fns = {"ours": (lambda: moe.moe_expert_gate_up(xp, D["W_gate"], D["W_up"], counts, offsets, h),
+                    lambda: moe.moe_expert_down(h, D["W_down"], counts, offsets, y)),
+           "grouped_mm": (lambda: F.grouped_mm(xp, wgu.transpose(1, 2), offs=ends),
+                          lambda: F.grouped_mm(h, D["W_down"].transpose(1, 2), offs=ends))}
+    try:
+        for f in fns["grouped_mm"]:
+            f()
+        torch.cuda.synchronize()
+    except Exception as e:  # a torch build without the grouped GEMM for this device
+        return {"unavailable": f"{type(e).__name__}: {str(e)[:120]}"}
+    times = {n: ([], []) for n in fns}
+    clk = Clocks(local)
+    clk.__enter__()
+    for _ in range(3):
+        for n, pair in fns.items():
+            for j, f in enumerate(pair):
+                time.sleep(0.5)
+                for _ in range(3):
+                    f()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                for _ in range(10):
+                    f()
+                e1.record()
+                torch.cuda.synchronize()
+                times[n][j].append(e0.elapsed_time(e1) / 10)
+    clk.__exit__(None, None, None)
+    med = {n: {"gate_up_ms": statistics.median(t[0]), "down_ms": statistics.median(t[1])} for n, t in times.items()}
+    del wgu, h, y
+    return {"vendor": "torch.nn.functional.grouped_mm", **med,
+            "ours_over_vendor_time": (med["ours"]["gate_up_ms"] + med["ours"]["down_ms"]) /
+                                     (med["grouped_mm"]["gate_up_ms"] + med["grouped_mm"]["down_ms"]),
+            "clocks": clk.summary(),
+            "note": "vendor gate/up writes g|u (2 d_ff columns) without the SwiGLU product"}
+
+
 def measure_workload(a, w, dev, world, rank, local, barrier, max_over_ranks, headline: bool) -> dict:
     """Everything the bench reports for one workload: the timed layer, its roofline fractions, the stage
     breakdown and dominant kernel, near-tie tokens, end-to-end throughput and the CPU oracle sample."""
@@ -568,6 +626,7 @@ def measure_workload(a, w, dev, world, rank, local, barrier, max_over_ranks, hea
          "layer_roofline": layer_roofline(w, active, ms_per_step, pk), "dominant_kernel": kroof,
          "stages_ms": stage_ms, "near_ties": near_ties(L), "config": config_of(w, world)}
     r["e2e"] = None if a.no_e2e else e2e_of(L, a, barrier, world, max_over_ranks)
+    r["vendor_anchor"] = None if (a.no_anchor or world > 1) else vendor_anchor(L, a, bufs, local)
     if headline:
         r.update(headline_extras(L, a, barrier, pk, ms_per_step, bufs, active))
     r["cpu_baseline"] = None
@@ -616,10 +675,10 @@ def run_ours(a, w):
                 "layer_roofline": h["layer_roofline"], "cpu_baseline": h["cpu_baseline"], "e2e": h["e2e"],
                 "gpu_launches": h["gpu_launches"], "clocks": h["clocks"], "stages_ms": h["stages_ms"],
                 "active_experts": h["active_experts"], "near_ties": h["near_ties"],
-                "masked_layout": h.get("masked_layout"), "fp8_layer": h.get("fp8_layer"), "ep_p2p": h.get("ep_p2p")}
+                "vendor_anchor": h.get("vendor_anchor"), "masked_layout": h.get("masked_layout"), "fp8_layer": h.get("fp8_layer"), "ep_p2p": h.get("ep_p2p")}
         if len(results) > 1:
             keep = ("ms_per_step", "tokens_per_s", "layer_roofline", "dominant_kernel", "stages_ms", "near_ties",
-                    "active_experts", "clocks", "gpu_launches", "e2e", "cpu_baseline", "config")
+                    "active_experts", "clocks", "gpu_launches", "e2e", "cpu_baseline", "vendor_anchor", "config")
             line["workloads"] = {n: {k: r[k] for k in keep} for n, r in results.items()}
         print(json.dumps(line), flush=True)
     if world > 1:
