@@ -358,13 +358,13 @@ class Layer:
         self.ws = torch.empty(moe.forward_workspace_bytes(self.D["x"], self.D["W_r"], self.D["W_gate"], self.out, k,
                                                           w.eps), dtype=torch.uint8, device=dev)
 
-    def step(self, x=None):
+    def step(self, x=None, out=None):
         import moe_layer_forward_b200 as moe
 
         D, w = self.D, self.w
         moe.moe_forward(D["x"] if x is None else x, D["gamma"], D["W_r"], D["b"], D["W_gate"], D["W_up"],
-                        D["W_down"], self.out, top_k=w.top_k, eps=w.eps, topk_idx=self.idx, topk_w=self.wt,
-                        ws=self.ws, dev_status=self.status)
+                        D["W_down"], self.out if out is None else out, top_k=w.top_k, eps=w.eps, topk_idx=self.idx,
+                        topk_w=self.wt, ws=self.ws, dev_status=self.status)
 
     def check_status(self, where: str):
         if self.status.item() != 0:
@@ -461,24 +461,59 @@ def staged(L, a, barrier, pk) -> tuple:
 
 
 def e2e_of(L, a, barrier, world, max_over_ranks) -> dict:
-    """The same layer through moe_forward with the step's input copied from pinned host memory and its
-    output read back to the host every step, inside the timed region."""
+    """The same layer through moe_forward with every step's input copied from pinned host memory and every
+    step's output copied back to pinned host memory and waited for by the host, inside the timed region.
+    The copies run on two copy streams with double-buffered device input and output, so step i+1's input
+    copy and step i-1's output copy overlap step i's layer; the host waits for each step's output one step
+    later, and the region ends when the last output has reached the host."""
     import torch
 
+    w = L.w
     x_host = L.I["x"].pin_memory()
-    out_host = torch.empty(L.out.shape, dtype=L.out.dtype).pin_memory()
-    x_dev = torch.empty_like(L.D["x"])
+    out_host = [torch.empty(L.out.shape, dtype=L.out.dtype).pin_memory() for _ in range(2)]
+    x_dev = [torch.empty_like(L.D["x"]) for _ in range(2)]
+    out_dev = [L.out, torch.empty_like(L.out)]
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()
+    in_done, comp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    for e in comp_done + out_done:  # every buffer starts free
+        e.record(comp)
 
-    def one():
-        x_dev.copy_(x_host, non_blocking=True)
-        L.step(x_dev)
-        out_host.copy_(L.out, non_blocking=True)
-        torch.cuda.current_stream().synchronize()  # the host reads this step's result
+    def run(n: int, start_event=None):
+        for i in range(n):
+            b = i % 2
+            s_in.wait_event(comp_done[b])  # the layer of step i-2 has read x_dev[b]
+            if start_event is not None and i == 0:
+                s_in.wait_event(start_event)
+            with torch.cuda.stream(s_in):
+                x_dev[b].copy_(x_host, non_blocking=True)
+            in_done[b].record(s_in)
+            comp.wait_event(in_done[b])
+            comp.wait_event(out_done[b])  # the output copy of step i-2 has read out_dev[b]
+            L.step(x_dev[b], out_dev[b])
+            comp_done[b].record(comp)
+            s_out.wait_event(comp_done[b])
+            with torch.cuda.stream(s_out):
+                out_host[b].copy_(out_dev[b], non_blocking=True)
+            out_done[b].record(s_out)
+            if i >= 1:
+                out_done[(i - 1) % 2].synchronize()  # the host has step i-1's result
+        comp.wait_event(out_done[(n - 1) % 2])
 
-    ms, _, _ = _timed(one, a.steps, a.warmup, barrier)
-    value, _ = aggregate(ms, L.w.T, a.steps, world, max_over_ranks)
+    run(a.warmup)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(comp)
+    run(a.steps, start_event=e0)
+    e1.record(comp)
+    barrier()
+    ms = e0.elapsed_time(e1)
+    L.check_status("in the end-to-end timing")
+    value, _ = aggregate(ms, w.T, a.steps, world, max_over_ranks)
     return {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
-            "d2h_bytes_per_step": out_host.numel() * out_host.element_size()}
+            "d2h_bytes_per_step": out_host[0].numel() * out_host[0].element_size(),
+            "copies": "pinned host memory, two copy streams, double-buffered; the host waits for every output"}
 
 
 def headline_extras(L, a, barrier, pk, ms_per_step, staged_bufs, active) -> dict:
