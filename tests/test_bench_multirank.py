@@ -106,3 +106,25 @@ def test_clock_summary_decodes_throttle_reasons():
     assert s["sm_mhz"] == 1650.0 and s["sm_min_mhz"] == 1400 and s["sm_max_mhz"] == 1965.0
     assert s["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
     assert s["samples"] == 4 and s["power_w"] == 970.0
+
+
+def test_layer_roofline_binds_decode_to_hbm_and_prefill_to_the_tensor_peak():
+    # the bench's layer fractions from the workloads' own sizes: decode streams the active experts' weights
+    # (HBM-bound), prefill runs 6 S d d_ff flops (tensor-bound); recomputed here from the shapes by hand
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+
+    pk = {"hbm_gbs": 6550.1, "bf16_tflops": 1640.7, "bf16_tflops_sustained": 1365.9, "source": "measured"}
+    dec = synth.WORKLOADS["decode"]
+    r = bench.layer_roofline(dec, 128, 0.7867, pk)
+    weights = 128 * 3 * 4096 * 1536 * 2
+    io = 128 * 4096 * (2 + 2) + 128 * 4096 * 4 + 4096 * 4 + 128 * 4
+    assert r["algorithmic_bytes"] == weights + io == 4836049408
+    assert r["bound"] == "hbm" and abs(r["frac"] - 4836049408 / 0.7867e-3 / 6550.1e9) < 1e-12
+    pre = synth.WORKLOADS["prefill"]
+    r = bench.layer_roofline(pre, 128, 2.5959, pk)
+    assert r["expert_flops"] == 6.0 * 8192 * 8 * 4096 * 1536
+    assert r["bound"] == "tensor" and abs(r["frac"] - 2.473901162496e12 / 2.5959e-3 / 1640.7e12) < 1e-12
+    assert abs(r["frac_sustained"] - 2.473901162496e12 / 2.5959e-3 / 1365.9e12) < 1e-12
+    assert abs(r["t_roof_ms"] - 2.473901162496e12 / 1640.7e12 * 1e3) < 1e-9
