@@ -447,6 +447,8 @@ moe_status_t moe_forward(const moe_shape_t* shape, const moe_weights_t* wts, con
     void* xp = fused_gather ? nullptr : cv.take((size_t)S * d * es);
     void* h = cv.take((size_t)S * d_ff * es);
     void* y = cv.take((size_t)S * d * es);
+    // the tile counter of the gate/up GEMM's dynamic schedule (two-row-block tiles), zeroed per call
+    int32_t* tile_ctr = static_cast<int32_t*>(cv.take(sizeof(int32_t)));
     bool query = false;
     st = check_ws(ws, ws_bytes, cv.off, &query);
     if (st != MOE_OK || query) return st;
@@ -463,6 +465,8 @@ moe_status_t moe_forward(const moe_shape_t* shape, const moe_weights_t* wts, con
         if (st != MOE_OK) return st;
     }
     if (T == 0) return MOE_OK;
+    st = cuda_status(cudaMemsetAsync(tile_ctr, 0, sizeof(int32_t), c.stream));
+    if (st != MOE_OK) return st;
     const int xdt = shape->x_dtype;
     // 1. RMSNorm: v rounded to the expert dtype, and 1/rms for the router
     st = cuda_status(launch_rmsnorm(c, x, xdt, wts->gamma, T, d, shape->eps, v, wdt, rstd));
@@ -480,7 +484,8 @@ moe_status_t moe_forward(const moe_shape_t* shape, const moe_weights_t* wts, con
     // 4. grouped SwiGLU MLP
     if (wdt == MOE_BF16) {
         st = cuda_status(launch_gate_up_bf16(c, fused_gather ? v : xp, wts->W_gate, wts->W_up, counts, offsets, S, E,
-                                             d, d_ff, h, dev_status, fused_gather ? slot_token : nullptr, T));
+                                             d, d_ff, h, dev_status, fused_gather ? slot_token : nullptr, T, 0, 0, false,
+                                             tile_ctr));
         if (st != MOE_OK) return st;
         st = cuda_status(launch_down_bf16(c, h, wts->W_down, counts, offsets, S, E, d, d_ff, y, dev_status));
     } else {

@@ -659,12 +659,15 @@ bool gate_up_needs_permuted_rows(int S, int E) { return use_pair_gemm(S, E, 256)
 
 cudaError_t launch_gate_up_bf16(const Ctx& c, const void* xp, const void* Wg, const void* Wu, const int32_t* counts,
                                 const int32_t* offsets, int S, int E, int d, int d_ff, void* h, int32_t* status,
-                                const int32_t* gather, int act_rows, int cap, int S_sel, bool raw) {
+                                const int32_t* gather, int act_rows, int cap, int S_sel, bool raw,
+                                int32_t* tile_ctr) {
     if (S == 0) return cudaSuccess;
     const int Ss = S_sel > 0 ? S_sel : S;  // rows the tile form is chosen for
     if (gather && (cap > 0 || gate_up_needs_permuted_rows(Ss, E))) return cudaErrorInvalidValue;
     if (cap == 0 && use_pair_gemm(Ss, E, 256))
         return launch_gate_up_bf16_pair(c, xp, Wg, Wu, counts, offsets, S, E, d, d_ff, h, status, raw);
+    if (cap == 0 && !gather && use_dual_gemm(Ss, E, 256))
+        return launch_gate_up_bf16_dual(c, xp, Wg, Wu, counts, offsets, S, E, d, d_ff, h, status, raw, tile_ctr);
     tc::Args a{counts, offsets, E, d, d_ff, static_cast<uint16_t*>(h), (int64_t)d_ff * (raw ? 2 : 1), status, gather,
                static_cast<const uint16_t*>(xp), cap, S, gather ? act_rows : 0};
     a.raw = raw ? 1 : 0;

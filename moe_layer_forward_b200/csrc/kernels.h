@@ -110,7 +110,7 @@ bool gate_up_needs_permuted_rows(int S, int E);
 cudaError_t launch_gate_up_bf16(const Ctx& c, const void* xp, const void* Wg, const void* Wu, const int32_t* counts,
                                 const int32_t* offsets, int S, int E, int d, int d_ff, void* h, int32_t* status,
                                 const int32_t* gather = nullptr, int act_rows = 0, int cap = 0, int S_sel = 0,
-                                bool raw = false);
+                                bool raw = false, int32_t* tile_ctr = nullptr);
 cudaError_t launch_down_bf16(const Ctx& c, const void* h, const void* Wd, const int32_t* counts, const int32_t* offsets,
                              int S, int E, int d, int d_ff, void* y, int32_t* status, int cap = 0, int S_sel = 0);
 // CTA-pair (cta_group::2) variants for experts with many rows each (expert_tc2.cu)
@@ -120,6 +120,13 @@ cudaError_t launch_gate_up_bf16_pair(const Ctx& c, const void* xp, const void* W
                                      void* h, int32_t* status, bool raw = false);
 cudaError_t launch_down_bf16_pair(const Ctx& c, const void* h, const void* Wd, const int32_t* counts,
                                   const int32_t* offsets, int S, int E, int d, int d_ff, void* y, int32_t* status);
+// Gate/up tiles of two 128-row blocks of one expert sharing each staged weight slice, one CTA
+// (expert_tc_dual.cu), for experts averaging 256 rows up to the CTA-pair range.  tile_ctr (one int, zero
+// before the launch) gives a dynamic schedule; null, CTA-strided tiles.
+bool use_dual_gemm(int S, int E, int n_out);
+cudaError_t launch_gate_up_bf16_dual(const Ctx& c, const void* xp, const void* Wg, const void* Wu,
+                                     const int32_t* counts, const int32_t* offsets, int S, int E, int d, int d_ff,
+                                     void* h, int32_t* status, bool raw, int32_t* tile_ctr);
 // Block-FP8 experts (expert_fp8.cu): E4M3 codes, fp32 scales per 128 x 128 weight block and per
 // (row, 128 columns) of a GEMM input
 cudaError_t launch_quant_fp8(const Ctx& c, const void* x, int dt, int64_t rows, int64_t cols, int blk_rows,

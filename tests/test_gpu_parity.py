@@ -447,6 +447,7 @@ SMALL = {
     # (T, d, E, d_ff, x, w, out): weights-as-M (few rows per expert) and rows-as-M (many)
     "decode_like": (96, 512, 64, 256, "bf16", "bf16", "bf16"),
     "prefill_like": (1200, 256, 8, 256, "bf16", "bf16", "bf16"),
+    "dual_like": (600, 256, 16, 256, "bf16", "bf16", "bf16"),  # ~300 rows per expert: two-row-block gate/up
     "block_like": (160, 256, 32, 384, "f32", "bf16", "f32"),
     "mixed_out": (50, 256, 16, 128, "f32", "bf16", "bf16"),
     "f32_experts": (40, 64, 16, 48, "bf16", "f32", "f32"),
@@ -488,7 +489,7 @@ def test_forward_workspace_too_small_is_rejected(moe):
     assert ei.value.status == 3
 
 
-@pytest.mark.parametrize("name", ["decode_like", "block_like", "prefill_like"])
+@pytest.mark.parametrize("name", ["decode_like", "block_like", "prefill_like", "dual_like"])
 def test_forward_replays_from_a_cuda_graph(moe, name):
     # the whole layer is capturable (no host sync, shape-only grids, caller-owned workspace): a graph
     # captured once replays the eager result bit for bit, and follows new data written into its input

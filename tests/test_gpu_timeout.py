@@ -47,6 +47,7 @@ def _stalled(moe, fn):
 GEMM_CASES = {
     "weights_as_m": (16, 4, 512, 256),
     "rows_as_m": (4, 100, 512, 256),
+    "row_block_pairs": (4, 300, 512, 256),
     "cta_pairs": (2, 800, 256, 256),
 }
 
@@ -104,10 +105,10 @@ def test_fp8_expert_gemms_time_out_and_recover(moe):
         assert torch.equal(a, b)
 
 
-@pytest.mark.parametrize("name", ["decode_like", "prefill_like"])
+@pytest.mark.parametrize("name", ["decode_like", "prefill_like", "dual_like"])
 def test_layer_times_out_and_the_next_call_matches_the_oracle(moe, name):
     # the whole layer: router logits and both expert GEMMs stall (with few rows per expert the gate/up GEMM
-    # gathers its rows in place; with many it runs on CTA pairs)
+    # gathers its rows in place; with ~300 it runs two-row-block tiles on a dynamic schedule; with many, CTA pairs)
     T, d, E, d_ff, xd, wd, od = SMALL[name]
     dt = {"bf16": torch.bfloat16, "f32": torch.float32}
     w = synth.Workload(name, T, d, E, d_ff, x_dtype=dt[xd], w_dtype=dt[wd], out_dtype=dt[od], seed=832)
