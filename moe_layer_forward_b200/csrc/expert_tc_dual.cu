@@ -1,29 +1,33 @@
-// Step 4 for experts of ~256-768 rows: grouped GEMMs whose tile is two 128-row blocks of one expert
+// Step 4, gate/up, for experts of ~256-767 rows: grouped GEMM tiles of two 128-row blocks of one expert
 // sharing each staged weight slice.
 //
 // Same mathematics as expert_tc.cu ("推理计算流梳理", §实际 MLP 计算策略 and §EP 路径):
-//   gate/up: h = SiLU(xp W_gate^T) ⊙ (xp W_up^T)        down: y = h W_down^T
-// The one-CTA 128 x 256 tile is bound by the traffic through shared memory:
-// per K = 16 step TMA writes 4 KB of token rows and 8 KB of weights and the MMA
-// reads them again, 24 KB per 1.05 MFLOP.  Here a tile is (expert e, row pair
-// rp = rows [256 rp, 256 rp + 256), column block cb): two MMAs per K step, one
-// per 128-row half, read the same staged weight slice into two accumulators,
-// so a K step moves 40 KB per 2.1 MFLOP (19 KB per MFLOP).  The two
-// accumulators fill all 512 TMEM columns, so a tile's accumulators are not
-// double-buffered: eight epilogue warps (one per TMEM lane quarter and half)
-// drain them, writing full 32-row chunks by TMA, before the next tile's
-// MMAs start; the producer keeps filling the stage ring meanwhile.  Row
-// padding is 128 rows, as in the one-CTA kernel: a pair whose second half has
-// no rows skips its loads and its MMAs.
+//   h = SiLU(xp W_gate^T) ⊙ (xp W_up^T)
+// At the burst clock the one-CTA 128 x 256 tile is paced by delivering its operands into shared memory,
+// two thirds of them weight bytes.  Here a tile is (expert e, row pair rp = rows [256 rp, 256 rp + 256),
+// column block cb): two MMAs per K step, one per 128-row half, read the same staged weight slice into two
+// accumulators, which halves the weight bytes per MMA.  Row padding stays 128 rows: a pair whose second half
+// has no rows skips its loads and its MMAs.
+//
+// The two accumulators fill all 512 TMEM columns, so they are single-buffered.  Eight epilogue warps (one
+// per TMEM lane quarter and half) read them one 32-column chunk ahead of their math and stores and release
+// them as soon as their last chunk has landed; full 32-row pieces leave by TMA.
+//
+// Schedule: with a tile counter (moe_forward passes one, zeroed per call) the producer takes the next
+// tile from it, so CTAs that drew light tiles (half-filled pairs) take more; without one, CTA i runs tiles
+// i, i + gridDim.x, ...  The producer writes tile j's id to ring1[j % 8] before arming the tile's first
+// stage (the barrier's arrive publishes it); the MMA warp reads it behind that stage's barrier and passes
+// it on in ring2[j % 4] behind tidb[j % 4] to the epilogue.  An id of -1 (no more tiles) travels the same
+// way on one stage armed with no data.
 //
 // Warp roles (1 CTA per SM, 320 threads):
-//   warp 0      TMA producer: a 3-stage ring of 64-wide K slices (token rows of
-//               both halves, the weight slice), 128-byte swizzle
+//   warp 0      TMA producer: a 3-stage ring of 64-wide K slices (token rows of both halves, the weight
+//               slice), 128-byte swizzle
 //   warp 1      owns the TMEM allocation; lane 0 issues the MMAs and commits
 //   warps 2..5  epilogue of the first half (TMEM lane quarters 2,3,0,1)
 //   warps 6..9  epilogue of the second half
-// Every wait is bounded; a wait that gives up raises DEV_TIMEOUT and all roles
-// unwind as in expert_tc.cu (drains bounded by time only, TMEM freed last).
+// Every wait is bounded; a wait that gives up raises DEV_TIMEOUT and all roles unwind as in expert_tc.cu
+// (drains bounded by time only, TMEM freed last).
 #include <cuda.h>
 #include <math.h>
 
