@@ -312,6 +312,20 @@ def _timed(fn, steps: int, warmup: int, barrier, clocks_gpu=None):
     return e0.elapsed_time(e1), (clk.summary() if clk else None), launches
 
 
+def gate_up_kernel_name(S: int, E: int) -> str:
+    """The gate/up GEMM form the library picks for S routed rows over E experts (the host's selection by
+    average rows per expert: weights-as-M up to 32, rows-as-M up to 255, two-row-block tiles up to 767, CTA
+    pairs above)."""
+    avg = S // E if E > 0 else 0
+    if avg >= 768:
+        return "grouped_gemm_2sm_kernel (expert gate/up + SwiGLU, CTA pairs)"
+    if avg >= 256:
+        return "grouped_gemm_dual_kernel (expert gate/up + SwiGLU, two 128-row blocks per tile)"
+    if avg > 32:
+        return "grouped_gemm_kernel (expert gate/up + SwiGLU, rows-as-M)"
+    return "grouped_gemm_kernel (expert gate/up + SwiGLU, weights-as-M)"
+
+
 def layer_roofline(w, active: int, ms: float, pk: dict) -> dict:
     """The whole layer against its binding roofline: algorithmic bytes (active experts' weights, X, R, W_r,
     gamma, b) over the measured copy peak, or expert-GEMM flops (6 S d d_ff) over the measured bf16 peak."""
@@ -452,7 +466,8 @@ def staged(L, a, barrier, pk) -> tuple:
         roof["traffic_note"] = ("DRAM bytes of the same kernel template as run by moe_forward, which gathers the "
                                 "token rows from V instead of reading the permuted copy Xp timed here (S*d*2 - "
                                 "T*d*2 fewer algorithmic bytes)")
-    roof["kernel"] = "grouped_gemm_kernel (expert gate/up + SwiGLU)"
+    roof["kernel"] = (gate_up_kernel_name(S, E) if w.w_dtype == torch.bfloat16
+                      else "fp32 expert kernel (expert_simt.cu, gate/up + SwiGLU)")
     roof["algorithmic_bytes_per_launch"] = gate_up_bytes
     roof["algorithmic_flops_per_launch"] = gate_up_flops
     roof["launch_ms"] = stage_ms["gate_up"]

@@ -128,3 +128,15 @@ def test_layer_roofline_binds_decode_to_hbm_and_prefill_to_the_tensor_peak():
     assert r["bound"] == "tensor" and abs(r["frac"] - 2.473901162496e12 / 2.5959e-3 / 1640.7e12) < 1e-12
     assert abs(r["frac_sustained"] - 2.473901162496e12 / 2.5959e-3 / 1365.9e12) < 1e-12
     assert abs(r["t_roof_ms"] - 2.473901162496e12 / 1640.7e12 * 1e3) < 1e-9
+
+
+def test_dominant_kernel_label_follows_the_tile_form_selection():
+    # the bench names the gate/up kernel the library selects by average rows per expert
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+
+    want = {"decode": "weights-as-M", "block": "rows-as-M", "prefill": "two 128-row blocks", "skewed": "CTA pairs"}
+    for name, form in want.items():
+        w = synth.WORKLOADS[name]
+        assert form in bench.gate_up_kernel_name(w.T * w.top_k, w.E), name
